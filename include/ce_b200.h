@@ -1,0 +1,199 @@
+/*
+ * ce_b200.h -- fused softmax cross-entropy on one NVIDIA B200 (sm_100a).
+ *
+ * C ABI. Plain pointers and sizes; no framework types. All device pointers
+ * refer to memory of the device that is current on the calling thread; the
+ * `cuda_stream` argument is a cudaStream_t (NULL = the legacy default stream).
+ *
+ * Ownership. The caller owns every buffer, the workspace and the stream. The
+ * library allocates no device memory per call and writes nothing but the
+ * outputs named in each call and the workspace handed to it. The one piece
+ * of library-owned device state is a per-device error word (see
+ * ce_get_error).
+ *
+ * Completion. Calls are asynchronous: they validate their arguments on the
+ * host, enqueue kernels on `cuda_stream` and return. Every output element is
+ * written on every call that returns CE_OK, including rows that are ignored
+ * (a stale buffer content never survives a successful call).
+ *
+ * Errors. Problems the host can see (a null pointer, a bad size, dtype or
+ * layout, an output overlapping an input, a short workspace) are returned as
+ * a status before anything is enqueued. A target outside [0, V) that is not
+ * ignore_index is only seen on the device: that row's loss (and, in the
+ * backward, its gradient row) is written as NaN and the device error word is
+ * set; ce_get_error reports it.
+ *
+ * Row addressing (ce_layout). Logical row r of an operand, 0 <= r < N, starts
+ * at element offset
+ *     (r / inner) * s_outer + (r % inner) * s_inner
+ * from the base pointer, and its column j sits a further j * s_col elements
+ * on. Offsets are in elements, 64-bit. A plain (N, V) matrix with row stride
+ * ld is {inner = N, s_outer = 0, s_inner = ld, s_col = 1}. A view x[:, :-1]
+ * of a (B, L, V) tensor is {inner = L - 1, s_outer = L*V, s_inner = V,
+ * s_col = 1} with N = B*(L-1); the matching targets t[:, 1:] of a (B, L)
+ * tensor are base t + 1 with {inner = L - 1, s_outer = L, s_inner = 1}.
+ * Views are read in place: the library never makes a contiguous copy (MLX
+ * issue #4686: the VJP went wrong through exactly such a hidden copy whose
+ * output aliased it). Loads are vectorised to 16 bytes when s_col = 1 and
+ * every row starts on a 16-byte boundary; other layouts take a scalar path.
+ *
+ * Rows are counted in 64 bits and every launch walks its rows in a
+ * grid-stride loop, so no grid dimension limits N (MLX PR #4776: a grid
+ * truncated past 2^32 threads silently skipped rows from 2^27 rows up).
+ */
+#ifndef CE_B200_H
+#define CE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { CE_F32 = 0, CE_BF16 = 1, CE_F16 = 2 } ce_dtype;
+typedef enum { CE_I32 = 0, CE_I64 = 1 } ce_index_dtype;
+
+typedef struct {
+    int64_t inner;   /* rows per outer block, >= 1 */
+    int64_t s_outer; /* element stride between outer blocks */
+    int64_t s_inner; /* element stride between rows of one block */
+    int64_t s_col;   /* element stride between columns (unused for targets) */
+} ce_layout;
+
+typedef enum {
+    CE_OK = 0,
+    CE_EINVAL = 1,     /* bad size, pointer, dtype or layout */
+    CE_EALIAS = 2,     /* an output overlaps an input (other than the allowed in-place) */
+    CE_EWORKSPACE = 3, /* workspace missing or smaller than the *_workspace_size query */
+    CE_ECUDA = 4,      /* a CUDA runtime call failed (launch, attribute query) */
+    CE_ETARGET = 5,    /* device flag: a target outside [0, V) that is not ignore_index */
+    CE_ENOTSUP = 6     /* a configuration this build does not implement */
+} ce_status;
+
+/* ------------------------------------------------------------------------ *
+ * Row cross-entropy over an (N, V) logits operand.
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of workspace ce_forward needs for this shape. Long rows on few rows
+ * are split across several CTAs whose partial (max, scaled sum) states are
+ * merged by a second launch; the workspace holds those partials. Returns 0
+ * when no split is used. `num_sms` is the device's multiprocessor count, or
+ * <= 0 to query the current device. */
+size_t ce_workspace_size(int64_t N, int64_t V, ce_dtype dt, int num_sms);
+
+/* Forward. For each row i with target y_i (ignore_index rows excepted):
+ *     m_i   = max_j z_ij
+ *     lse_i = m_i + log sum_j exp(z_ij - m_i)            (online, one pass)
+ *     loss_i = (lse_i - m_i) - (1 - eps)(z_i,y_i - m_i) - eps (mean_j z_ij - m_i)
+ * i.e. (1-eps)(lse - z_y) + eps(lse - mean z), assembled from max-shifted
+ * values so that the gaps between logits survive at any magnitude.
+ * Sources: Ineshin, "A fused linear cross-entropy forward kernel for Apple
+ * GPUs", section 1 (the running (m, s) state and logsumexp = m + log s);
+ * MLX PR #4188 "Shift by the max in cross_entropy" (the shifted assembly and
+ * the label-smoothing term, which subtracts the mean logit).
+ *
+ * logits   N x V values of dtype `dt`, addressed through `lg`.
+ * targets  N class indices of type `tdt`, addressed through `tg` (column 0).
+ * label_smoothing  eps in [0, 1]; eps/V goes to every class.
+ * ignore_index     rows whose target equals it get loss 0 (lse still written).
+ * loss     N floats, contiguous. Out-of-range target: NaN (and the error word).
+ * lse      N floats, contiguous: lse_i rounded to float.
+ * lse_lo   N floats or NULL: lse_i minus the float `lse_i`, rounded to float
+ *          (the pair carries lse to about 48 bits; ce_backward uses it to keep
+ *          the softmax exact when |logits| is so large that float lse loses
+ *          the gap, e.g. equal logits at 1e8).
+ * argmax   N int32 or NULL: the lowest index attaining the row max (the first
+ *          NaN if the row has one).
+ * workspace, ws_bytes  at least ce_workspace_size(N, V, dt, sms) bytes,
+ *          16-byte aligned; may be NULL when that size is 0.
+ * Special rows: an all -inf row gives lse = -inf and loss NaN; a NaN in the
+ * row gives lse and loss NaN.
+ * Outputs must not overlap each other, the logits or the targets. */
+ce_status ce_forward(const void* logits, ce_dtype dt, ce_layout lg,
+                     int64_t N, int64_t V,
+                     const void* targets, ce_index_dtype tdt, ce_layout tg,
+                     float label_smoothing, int64_t ignore_index,
+                     float* loss, float* lse, float* lse_lo, int32_t* argmax,
+                     void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* Backward (VJP of sum_i g_i loss_i with respect to the logits):
+ *     dz_ij = g_i (exp(z_ij - lse_i) - (1 - eps)[j = y_i] - eps/V)
+ * from the saved lse (and lse_lo when given); ignore_index rows get a zero
+ * row, out-of-range targets a NaN row and the error word.
+ * Sources: MLX issue #4686 (the fast.cross_entropy VJP, including the strided
+ * view x[:, :-1]); Ineshin section 1 (the backward regenerates what it needs
+ * from the saved log-sum-exp).
+ *
+ * grad_out     g: N floats read at grad_out[i * grad_stride]; grad_stride = 0
+ *              broadcasts one scalar (e.g. 1/count for a mean reduction).
+ * lse, lse_lo  as written by ce_forward (lse_lo may be NULL: taken as 0).
+ * dlogits      N x V values of dtype `ddt` through layout `dl`. It may be the
+ *              logits themselves (same pointer, same dtype, same layout:
+ *              each element is read before it is overwritten by the same
+ *              thread); any other overlap with an input is CE_EALIAS. */
+ce_status ce_backward(const float* grad_out, int64_t grad_stride,
+                      const void* logits, ce_dtype dt, ce_layout lg,
+                      int64_t N, int64_t V,
+                      const void* targets, ce_index_dtype tdt, ce_layout tg,
+                      const float* lse, const float* lse_lo,
+                      float label_smoothing, int64_t ignore_index,
+                      void* dlogits, ce_dtype ddt, ce_layout dl,
+                      void* cuda_stream);
+
+/* ------------------------------------------------------------------------ *
+ * Fused-linear cross-entropy: logits Z = H W^T are never stored.
+ * Source: Ineshin, "A fused linear cross-entropy forward kernel for Apple
+ * GPUs", section 1 (Z = H W^T streamed over vocabulary tiles into the running
+ * (m, s) state, the target logit captured when its tile passes; the backward
+ * regenerates the logits tile by tile from the saved log-sum-exp).
+ * H: N x D bf16, row stride ld_h elements; W: V x D bf16, row stride ld_w.
+ * D must be a multiple of 64 and ld_h, ld_w multiples of 8 (16-byte rows for
+ * the tensor-memory-access engine); H and W 16-byte aligned.
+ * ------------------------------------------------------------------------ */
+
+/* Workspace bytes for linear_ce_forward (per-row partial states of the
+ * vocabulary splits). `num_sms` <= 0 queries the current device. */
+size_t linear_ce_workspace_size(int64_t N, int64_t V, int64_t D, int num_sms);
+
+/* loss and lse of Z = H W^T rows, same definitions as ce_forward.
+ * targets: N indices of type tdt, contiguous. loss, lse: N floats. */
+ce_status linear_ce_forward(const void* H, int64_t ld_h, const void* W, int64_t ld_w,
+                            const void* targets, ce_index_dtype tdt,
+                            int64_t N, int64_t V, int64_t D,
+                            float label_smoothing, int64_t ignore_index,
+                            float* loss, float* lse,
+                            void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* Workspace bytes for linear_ce_backward (one vocabulary chunk of the
+ * gradient of the logits in both orientations, transposed copies of H and
+ * W, and the float dH accumulator). */
+size_t linear_ce_backward_workspace_size(int64_t N, int64_t V, int64_t D, int num_sms);
+
+/* dH = G W and dW = G^T H with G_ij = g_i (exp(Z_ij - lse_i) - (1-eps)[j=y_i]
+ * - eps/V), Z recomputed chunk by chunk of the vocabulary from H and W and
+ * the saved lse. dH: N x D, dW: V x D, contiguous, dtype CE_BF16 or CE_F32
+ * (accumulation is float either way). */
+ce_status linear_ce_backward(const float* grad_out, int64_t grad_stride,
+                             const void* H, int64_t ld_h, const void* W, int64_t ld_w,
+                             const void* targets, ce_index_dtype tdt, const float* lse,
+                             int64_t N, int64_t V, int64_t D,
+                             float label_smoothing, int64_t ignore_index,
+                             void* dH, ce_dtype dH_dt, void* dW, ce_dtype dW_dt,
+                             void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* ------------------------------------------------------------------------ */
+
+/* Waits for `cuda_stream`, then reads and clears the current device's error
+ * word: CE_ETARGET if any launch since the last call saw an out-of-range
+ * target, CE_ECUDA if the wait itself failed, CE_OK otherwise. */
+ce_status ce_get_error(void* cuda_stream);
+
+/* Static text for a status code. */
+const char* ce_status_string(ce_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CE_B200_H */

@@ -1,0 +1,359 @@
+// C ABI of the fused softmax cross-entropy library: argument validation,
+// workspace sizing, kernel planning and launches. No allocation, no
+// synchronisation on the hot path.
+#include <mutex>
+
+#include "ce_b200.h"
+#include "ce_launch.h"
+#include "ce_linear.h"
+
+namespace ceb {
+
+// One error word per device; kernels receive its address as an argument.
+static __device__ unsigned int g_ce_error_word;
+
+static constexpr int kMaxDevices = 64;
+static std::mutex g_dev_mutex;
+static unsigned int* g_err_ptr[kMaxDevices];
+static int g_num_sms[kMaxDevices];
+
+static int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
+unsigned int* error_word() {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!g_err_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_ce_error_word) != cudaSuccess) return nullptr;
+        g_err_ptr[dev] = static_cast<unsigned int*>(p);
+    }
+    return g_err_ptr[dev];
+}
+
+int device_sms(int num_sms) {
+    if (num_sms > 0) return num_sms;
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!g_num_sms[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        g_num_sms[dev] = n;
+    }
+    return g_num_sms[dev];
+}
+
+int elem_size(int dt) { return dt == CE_F32 ? 4 : 2; }
+
+// Byte range [lo, hi) that a layout can touch for N rows of V columns: a
+// conservative box over the outer, inner and column index ranges.
+struct Extent {
+    uintptr_t lo, hi;
+};
+
+static Extent layout_extent(const void* base, const Layout& L, int64_t N, int64_t V, int esz) {
+    const int64_t nouter = (N + L.inner - 1) / L.inner;
+    const int64_t ninner = N < L.inner ? N : L.inner;
+    int64_t mn = 0, mx = 0;
+    auto span = [&](int64_t count, int64_t stride) {
+        if (count <= 1) return;
+        const int64_t d = (count - 1) * stride;
+        if (d < 0) mn += d; else mx += d;
+    };
+    span(nouter, L.s_outer);
+    span(ninner, L.s_inner);
+    span(V, L.s_col);
+    const uintptr_t b = reinterpret_cast<uintptr_t>(base);
+    return {b + (uintptr_t)(mn * esz), b + (uintptr_t)((mx + 1) * esz)};
+}
+
+static Extent flat_extent(const void* base, int64_t count, int esz) {
+    const uintptr_t b = reinterpret_cast<uintptr_t>(base);
+    return {b, b + (uintptr_t)(count * esz)};
+}
+
+static bool overlap(const Extent& a, const Extent& b) { return a.lo < b.hi && b.lo < a.hi; }
+
+// True when every row starts on a 16-byte boundary and columns are unit-stride.
+static bool vectorizable(const void* base, const Layout& L, int64_t N, int esz) {
+    if (L.s_col != 1) return false;
+    if (reinterpret_cast<uintptr_t>(base) % 16) return false;
+    if (N > L.inner && (L.s_outer * esz) % 16) return false;
+    if (N > 1 && L.inner > 1 && (L.s_inner * esz) % 16) return false;
+    return true;
+}
+
+static Layout to_layout(const ce_layout& l) { return Layout{l.inner, l.s_outer, l.s_inner, l.s_col}; }
+
+static bool layout_ok(const ce_layout& l) { return l.inner >= 1; }
+
+// ---- forward planning --------------------------------------------------------
+static constexpr int kPackedMaxRowBytes = 4096;
+static constexpr int64_t kMinSplitVecs = 2048;  // one full step of a 512-thread CTA x 4 vectors
+
+static int packed_lanes(int64_t nvec) {
+    int G = 1;
+    while (G < 32 && nvec > 8 * (int64_t)G) G *= 2;
+    return G;
+}
+
+static bool use_packed(int64_t V, int esz) { return V * esz <= kPackedMaxRowBytes; }
+
+// Number of vocabulary splits per row for the CTA kernel: the smallest power
+// of two whose unit count fills the machine's CTA slots to >= 90% in the last
+// wave, keeping every split at least one full CTA step long.
+static int plan_splits(int64_t N, int64_t V, int esz, int sms) {
+    if (use_packed(V, esz) || N <= 0) return 1;
+    const int64_t nvec = V / (16 / esz);
+    const int64_t slots = (int64_t)sms * 2;
+    const int64_t max_splits = nvec / kMinSplitVecs > 1 ? nvec / kMinSplitVecs : 1;
+    int best = 1;
+    double best_eff = -1.0;
+    for (int64_t s = 1; s <= 256 && s <= max_splits; s *= 2) {
+        const int64_t units = N * s;
+        const int64_t waves = (units + slots - 1) / slots;
+        const double eff = (double)units / (double)(waves * slots);
+        if (eff >= 0.9) return (int)s;
+        if (eff > best_eff + 1e-9) {
+            best_eff = eff;
+            best = (int)s;
+        }
+    }
+    return best;
+}
+
+static FwdPlan plan_forward(int64_t N, int64_t V, int esz, bool vec_ok, int sms) {
+    FwdPlan p{};
+    const int vecw = 16 / esz;
+    p.vec = vec_ok ? vecw : 1;
+    p.splits = 1;
+    p.vec_per_split = 0;
+    if (use_packed(V, esz) || (!vec_ok && V <= 256)) {
+        p.kind = FwdPlan::kPacked;
+        const int64_t nvec = V / p.vec;
+        p.G = packed_lanes(nvec);
+        p.U = (p.G == 1 && nvec <= 2) ? 2 : 8;
+        const int64_t rows_per_block = 8 * (32 / p.G);
+        const int64_t want = (N + rows_per_block - 1) / rows_per_block;
+        const int64_t cap = (int64_t)sms * 16;
+        p.grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
+        return p;
+    }
+    p.kind = FwdPlan::kCta;
+    p.splits = plan_splits(N, V, esz, sms);
+    const int64_t nvec = V / p.vec;
+    int64_t vps = (nvec + p.splits - 1) / p.splits;
+    if (vps < 1) vps = 1;
+    p.splits = (int)((nvec + vps - 1) / vps);
+    if (p.splits < 1) p.splits = 1;
+    p.vec_per_split = vps;
+    const int64_t units = N * p.splits;
+    const int64_t cap = (int64_t)sms * 2;
+    p.grid = (int)(units < cap ? units : cap);
+    const int64_t mg = (N + 255) / 256;
+    p.merge_grid = (int)(mg < (int64_t)sms * 8 ? mg : (int64_t)sms * 8);
+    if (p.merge_grid < 1) p.merge_grid = 1;
+    return p;
+}
+
+static size_t forward_workspace(int64_t N, int64_t V, int esz, int sms) {
+    const int splits = plan_splits(N, V, esz, sms);
+    if (splits <= 1) return 0;
+    // the realised split count can only shrink (vectors per split rounded up)
+    return (size_t)splits * (size_t)N * sizeof(float4);
+}
+
+// ---- backward planning -------------------------------------------------------
+static constexpr int64_t kBwdChunkVecs = 2048;
+
+static BwdPlan plan_backward(int64_t N, int64_t V, int esz_in, bool vec_ok, int sms,
+                             int64_t* nchunks, int64_t* vpc) {
+    BwdPlan p{};
+    p.vec = vec_ok ? 16 / esz_in : 1;
+    const int64_t nvec = V / p.vec;
+    if (nvec <= 256) {
+        p.G = packed_lanes(nvec);
+        p.U = (p.G == 1 && nvec <= 2) ? 2 : 8;
+        *nchunks = 1;
+        *vpc = nvec > 0 ? nvec : 1;
+    } else {
+        p.G = 32;
+        p.U = 4;
+        *vpc = kBwdChunkVecs;
+        *nchunks = (nvec + kBwdChunkVecs - 1) / kBwdChunkVecs;
+    }
+    const int64_t groups_per_block = 256 / p.G;
+    const int64_t want = (N * *nchunks + groups_per_block - 1) / groups_per_block;
+    const int64_t cap = (int64_t)sms * 16;
+    p.grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
+    return p;
+}
+
+}  // namespace ceb
+
+using namespace ceb;
+
+extern "C" {
+
+size_t ce_workspace_size(int64_t N, int64_t V, ce_dtype dt, int num_sms) {
+    if (N <= 0 || V <= 0 || (dt != CE_F32 && dt != CE_BF16 && dt != CE_F16)) return 0;
+    return forward_workspace(N, V, elem_size(dt), device_sms(num_sms));
+}
+
+ce_status ce_forward(const void* logits, ce_dtype dt, ce_layout lg, int64_t N, int64_t V,
+                     const void* targets, ce_index_dtype tdt, ce_layout tg,
+                     float label_smoothing, int64_t ignore_index,
+                     float* loss, float* lse, float* lse_lo, int32_t* argmax,
+                     void* workspace, size_t ws_bytes, void* cuda_stream) {
+    if (N < 0 || V < 1 || V > INT32_MAX) return CE_EINVAL;
+    if (dt != CE_F32 && dt != CE_BF16 && dt != CE_F16) return CE_EINVAL;
+    if (tdt != CE_I32 && tdt != CE_I64) return CE_EINVAL;
+    if (!(label_smoothing >= 0.f && label_smoothing <= 1.f)) return CE_EINVAL;
+    if (N == 0) return CE_OK;
+    if (!logits || !targets || !loss || !lse) return CE_EINVAL;
+    if (!layout_ok(lg) || !layout_ok(tg)) return CE_EINVAL;
+    const int esz = elem_size(dt);
+    const int tsz = tdt == CE_I32 ? 4 : 8;
+    const Layout L = to_layout(lg), T = to_layout(tg);
+
+    // outputs must not overlap inputs or each other
+    const Extent ez = layout_extent(logits, L, N, V, esz);
+    const Extent et = layout_extent(targets, Layout{T.inner, T.s_outer, T.s_inner, 0}, N, 1, tsz);
+    Extent outs[4];
+    int nout = 0;
+    outs[nout++] = flat_extent(loss, N, 4);
+    outs[nout++] = flat_extent(lse, N, 4);
+    if (lse_lo) outs[nout++] = flat_extent(lse_lo, N, 4);
+    if (argmax) outs[nout++] = flat_extent(argmax, N, 4);
+    for (int i = 0; i < nout; ++i) {
+        if (overlap(outs[i], ez) || overlap(outs[i], et)) return CE_EALIAS;
+        for (int j = 0; j < i; ++j)
+            if (overlap(outs[i], outs[j])) return CE_EALIAS;
+    }
+
+    const int sms = device_sms(0);
+    const bool vec_ok = vectorizable(logits, L, N, esz);
+    FwdPlan plan = plan_forward(N, V, esz, vec_ok, sms);
+    FwdArgs a{};
+    if (plan.kind == FwdPlan::kCta && plan.splits > 1) {
+        const size_t need = (size_t)plan.splits * (size_t)N * sizeof(float4);
+        if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) % 16))
+            return CE_EWORKSPACE;
+        const Extent ew = flat_extent(workspace, (int64_t)need, 1);
+        if (overlap(ew, ez) || overlap(ew, et)) return CE_EALIAS;
+        for (int i = 0; i < nout; ++i)
+            if (overlap(ew, outs[i])) return CE_EALIAS;
+        a.part = static_cast<float4*>(workspace);
+    }
+    a.z = logits;
+    a.N = N;
+    a.V = V;
+    a.y = targets;
+    a.tdt = tdt == CE_I32 ? 0 : 1;
+    a.eps = label_smoothing;
+    a.ignore = ignore_index;
+    a.loss = loss;
+    a.lse = lse;
+    a.lse_lo = lse_lo;
+    a.argmax = argmax;
+    a.err = error_word();
+    if (!a.err) return CE_ECUDA;
+    a.splits = plan.splits;
+    a.vec_is_scalar = plan.vec == 1;
+    a.vec_per_split = plan.vec_per_split;
+    a.lz = L;
+    a.ly = T;
+    cudaError_t e = launch_forward(plan, a, (int)dt, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? CE_OK : CE_ECUDA;
+}
+
+ce_status ce_backward(const float* grad_out, int64_t grad_stride, const void* logits,
+                      ce_dtype dt, ce_layout lg, int64_t N, int64_t V, const void* targets,
+                      ce_index_dtype tdt, ce_layout tg, const float* lse, const float* lse_lo,
+                      float label_smoothing, int64_t ignore_index, void* dlogits, ce_dtype ddt,
+                      ce_layout dl, void* cuda_stream) {
+    if (N < 0 || V < 1 || V > INT32_MAX) return CE_EINVAL;
+    if (dt != CE_F32 && dt != CE_BF16 && dt != CE_F16) return CE_EINVAL;
+    if (ddt != CE_F32 && ddt != dt) return CE_ENOTSUP;
+    if (tdt != CE_I32 && tdt != CE_I64) return CE_EINVAL;
+    if (!(label_smoothing >= 0.f && label_smoothing <= 1.f)) return CE_EINVAL;
+    if (N == 0) return CE_OK;
+    if (!grad_out || !logits || !targets || !lse || !dlogits) return CE_EINVAL;
+    if (!layout_ok(lg) || !layout_ok(tg) || !layout_ok(dl)) return CE_EINVAL;
+    const int esz = elem_size(dt), dsz = elem_size(ddt);
+    const int tsz = tdt == CE_I32 ? 4 : 8;
+    const Layout L = to_layout(lg), T = to_layout(tg), D = to_layout(dl);
+
+    const Extent ez = layout_extent(logits, L, N, V, esz);
+    const Extent ed = layout_extent(dlogits, D, N, V, dsz);
+    const Extent et = layout_extent(targets, Layout{T.inner, T.s_outer, T.s_inner, 0}, N, 1, tsz);
+    const Extent eg = grad_stride == 0 ? flat_extent(grad_out, 1, 4)
+                                       : layout_extent(grad_out, Layout{N, 0, grad_stride, 0}, N, 1, 4);
+    const Extent el = flat_extent(lse, N, 4);
+    const bool in_place = dlogits == logits && ddt == dt && L.inner == D.inner &&
+                          L.s_outer == D.s_outer && L.s_inner == D.s_inner && L.s_col == D.s_col;
+    if (!in_place && overlap(ed, ez)) return CE_EALIAS;
+    if (overlap(ed, et) || overlap(ed, eg) || overlap(ed, el)) return CE_EALIAS;
+    if (lse_lo && overlap(ed, flat_extent(lse_lo, N, 4))) return CE_EALIAS;
+
+    const int sms = device_sms(0);
+    // vector path: both operands row-aligned with unit column stride
+    const bool vec_ok = vectorizable(logits, L, N, esz) && vectorizable(dlogits, D, N, dsz);
+    int64_t nchunks = 1, vpc = 1;
+    BwdPlan plan = plan_backward(N, V, esz, vec_ok, sms, &nchunks, &vpc);
+    BwdArgs a{};
+    a.g = grad_out;
+    a.g_stride = grad_stride;
+    a.z = logits;
+    a.N = N;
+    a.V = V;
+    a.y = targets;
+    a.tdt = tdt == CE_I32 ? 0 : 1;
+    a.lse = lse;
+    a.lse_lo = lse_lo;
+    a.eps = label_smoothing;
+    a.ignore = ignore_index;
+    a.dz = dlogits;
+    a.err = error_word();
+    if (!a.err) return CE_ECUDA;
+    a.nchunks = nchunks;
+    a.vec_per_chunk = vpc;
+    a.lz = L;
+    a.ly = T;
+    a.ld = D;
+    cudaError_t e = launch_backward(plan, a, (int)dt, (int)ddt, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? CE_OK : CE_ECUDA;
+}
+
+ce_status ce_get_error(void* cuda_stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess) return CE_ECUDA;
+    unsigned int w = 0;
+    if (cudaMemcpyFromSymbol(&w, g_ce_error_word, sizeof(w)) != cudaSuccess) return CE_ECUDA;
+    if (w) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_ce_error_word, &zero, sizeof(zero)) != cudaSuccess) return CE_ECUDA;
+        return CE_ETARGET;
+    }
+    return CE_OK;
+}
+
+const char* ce_status_string(ce_status s) {
+    switch (s) {
+        case CE_OK: return "ok";
+        case CE_EINVAL: return "invalid argument (size, pointer, dtype or layout)";
+        case CE_EALIAS: return "an output overlaps an input";
+        case CE_EWORKSPACE: return "workspace missing, misaligned or too small";
+        case CE_ECUDA: return "CUDA runtime error";
+        case CE_ETARGET: return "a target outside [0, V) that is not ignore_index";
+        case CE_ENOTSUP: return "configuration not supported";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,322 @@
+// Device-side building blocks of the row cross-entropy kernels (sm_100a).
+//
+// The per-row statistic is the online log-sum-exp state of Ineshin, "A fused
+// linear cross-entropy forward kernel for Apple GPUs", section 1: a running
+// maximum m and the sum s of exp(z - m), rescaled whenever m grows. We carry
+// two more numbers so the loss can be assembled from max-shifted values as in
+// MLX PR #4188 ("Shift by the max in cross_entropy"): t, the sum of (z - m)
+// over the k elements seen so far (the label-smoothing term needs the mean
+// logit, and the mean moves with the shift), and k itself.
+//
+// Merging two states is associative and is done with one operator everywhere
+// (lane shuffles, the one shared-memory exchange per CTA, the split merge):
+//   (m1,s1,t1,k1) + (m2,s2,t2,k2) = (M, s1 e^{m1-M} + s2 e^{m2-M},
+//                                    t1 + k1 (m1-M) + t2 + k2 (m2-M), k1+k2)
+// with M = max(m1, m2). A side whose m equals M takes factor 1 and shift 0, so
+// an empty side (m = -inf) merges as the identity and never produces
+// exp(-inf - (-inf)) = NaN.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ce_launch.h"
+
+namespace ceb {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Element offset of logical row r. A plain matrix (one outer block) needs no
+// division.
+__device__ __forceinline__ int64_t row_offset(const Layout& L, int64_t r, int64_t N) {
+    if (L.inner >= N) return r * L.s_inner;
+    const int64_t o = r / L.inner;
+    return o * L.s_outer + (r - o * L.inner) * L.s_inner;
+}
+
+// Hardware base-2 exponential (MUFU); exp(x) = ex2(x * log2 e).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// ---------------------------------------------------------------------------
+// Loads. VEC = 16 / sizeof(T) elements per 16-byte load on the vector path,
+// VEC = 1 on the scalar path. Streaming loads (evict-first) for data read once.
+template <typename T> struct ElemTraits;
+template <> struct ElemTraits<float> { static constexpr int kVec = 4; };
+template <> struct ElemTraits<__nv_bfloat16> { static constexpr int kVec = 8; };
+template <> struct ElemTraits<__half> { static constexpr int kVec = 8; };
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
+
+template <typename T>
+__device__ __forceinline__ void unpack_words(const uint4& r, float* out);
+
+template <>
+__device__ __forceinline__ void unpack_words<float>(const uint4& r, float* out) {
+    out[0] = __uint_as_float(r.x);
+    out[1] = __uint_as_float(r.y);
+    out[2] = __uint_as_float(r.z);
+    out[3] = __uint_as_float(r.w);
+}
+
+template <>
+__device__ __forceinline__ void unpack_words<__nv_bfloat16>(const uint4& r, float* out) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        out[2 * k] = __uint_as_float(w[k] << 16);
+        out[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    }
+}
+
+template <>
+__device__ __forceinline__ void unpack_words<__half>(const uint4& r, float* out) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        __half2 h = *reinterpret_cast<const __half2*>(&w[k]);
+        float2 f = __half22float2(h);
+        out[2 * k] = f.x;
+        out[2 * k + 1] = f.y;
+    }
+}
+
+// Loads VEC consecutive (VEC > 1, s_col = 1, 16-byte aligned) or one
+// (VEC = 1, any stride) element(s) starting at column `col` of `row`.
+template <typename T, int VEC>
+__device__ __forceinline__ void load_vec(const T* row, int64_t col, int64_t s_col, float* out) {
+    if constexpr (VEC == 1) {
+        out[0] = to_f32(row[col * s_col]);
+    } else {
+        const uint4 r = __ldcs(reinterpret_cast<const uint4*>(row + col));
+        unpack_words<T>(r, out);
+    }
+}
+
+// Plain (coherent) loads for kernels whose output may alias the input.
+template <typename T, int VEC>
+__device__ __forceinline__ void load_vec_coherent(const T* row, int64_t col, int64_t s_col,
+                                                  float* out) {
+    if constexpr (VEC == 1) {
+        out[0] = to_f32(row[col * s_col]);
+    } else {
+        const uint4 r = *reinterpret_cast<const uint4*>(row + col);
+        unpack_words<T>(r, out);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Stores of n = VEC floats converted to T (round to nearest even).
+__device__ __forceinline__ void cvt_store1(float* p, float v) { __stcs(p, v); }
+__device__ __forceinline__ void cvt_store1(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+__device__ __forceinline__ void cvt_store1(__half* p, float v) { *p = __float2half_rn(v); }
+
+__device__ __forceinline__ uint32_t pack2(__nv_bfloat16*, float a, float b) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack2(__half*, float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <typename TO, int VEC>
+__device__ __forceinline__ void store_vec(TO* row, int64_t col, int64_t s_col, const float* v) {
+    if constexpr (VEC == 1) {
+        cvt_store1(row + col * s_col, v[0]);
+    } else if constexpr (sizeof(TO) == 4) {
+        // VEC floats = VEC*4 bytes: one or two 16-byte stores
+#pragma unroll
+        for (int q = 0; q < VEC / 4; ++q) {
+            uint4 w = make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                                 __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+            __stcs(reinterpret_cast<uint4*>(row + col) + q, w);
+        }
+    } else {
+        static_assert(VEC == 8, "16-bit outputs are stored 8 at a time");
+        uint4 w = make_uint4(pack2((TO*)nullptr, v[0], v[1]), pack2((TO*)nullptr, v[2], v[3]),
+                             pack2((TO*)nullptr, v[4], v[5]), pack2((TO*)nullptr, v[6], v[7]));
+        __stcs(reinterpret_cast<uint4*>(row + col), w);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Online state.
+struct OnlineState {
+    float m;  // running max (never NaN: fmaxf drops NaN operands)
+    float s;  // sum of exp(z - m)
+    float t;  // sum of (z - m)
+    int k;    // elements seen
+    float av; // argmax value (NaN beats everything; first NaN wins)
+    int ai;   // argmax index, -1 = empty
+};
+
+__device__ __forceinline__ OnlineState empty_state() {
+    OnlineState st;
+    st.m = -INFINITY;
+    st.s = 0.f;
+    st.t = 0.f;
+    st.k = 0;
+    st.av = -INFINITY;
+    st.ai = -1;
+    return st;
+}
+
+// True when candidate (bv, bi) should replace (av, ai) as the argmax: a NaN
+// beats any number, a larger value wins, and equal values (or two NaNs) go to
+// the lower index.
+__device__ __forceinline__ bool argmax_better(float bv, int bi, float av, int ai) {
+    if (bi < 0) return false;
+    if (ai < 0) return true;
+    const bool bn = bv != bv, an = av != av;
+    if (bn != an) return bn;
+    if (!bn && bv != av) return bv > av;
+    return bi < ai;
+}
+
+// Rescale the state to a new max mn >= st.m.
+__device__ __forceinline__ void rescale_to(OnlineState& st, float mn) {
+    if (st.m != mn) {
+        st.s *= ex2((st.m - mn) * kLog2e);  // st.m = -inf gives 0
+        if (st.k != 0) st.t += (float)st.k * (st.m - mn);
+        st.m = mn;
+    }
+}
+
+// Folds n values (all valid) into the state: one max, one rescale, then one
+// exponential per element. Columns are col0 + i*dcol (used for argmax only).
+template <int n, bool ARGMAX>
+__device__ __forceinline__ void fold(OnlineState& st, const float* v, int col0, int dcol) {
+    float cm = v[0];
+#pragma unroll
+    for (int i = 1; i < n; ++i) cm = fmaxf(cm, v[i]);
+    rescale_to(st, fmaxf(st.m, cm));
+    const float ms = (st.m == -INFINITY) ? 0.f : st.m;
+    float sa = 0.f, ta = 0.f;
+#pragma unroll
+    for (int i = 0; i < n; ++i) {
+        const float d = v[i] - ms;
+        sa += ex2(d * kLog2e);
+        ta += d;
+    }
+    st.s += sa;
+    st.t += ta;
+    st.k += n;
+    if constexpr (ARGMAX) {
+#pragma unroll
+        for (int i = 0; i < n; ++i) {
+            const float x = v[i];
+            const bool take = (st.ai < 0) | (x > st.av) | ((x != x) & (st.av == st.av));
+            if (take) {
+                st.av = x;
+                st.ai = col0 + i * dcol;
+            }
+        }
+    }
+}
+
+template <bool ARGMAX>
+__device__ __forceinline__ void merge(OnlineState& a, const OnlineState& b) {
+    const float M = fmaxf(a.m, b.m);
+    const float fa = (a.m == M) ? 1.f : ex2((a.m - M) * kLog2e);
+    const float fb = (b.m == M) ? 1.f : ex2((b.m - M) * kLog2e);
+    const float ta = (a.k == 0 || a.m == M) ? 0.f : (float)a.k * (a.m - M);
+    const float tb = (b.k == 0 || b.m == M) ? 0.f : (float)b.k * (b.m - M);
+    a.s = a.s * fa + b.s * fb;
+    a.t = (a.t + ta) + (b.t + tb);
+    a.k += b.k;
+    a.m = M;
+    if constexpr (ARGMAX) {
+        if (argmax_better(b.av, b.ai, a.av, a.ai)) {
+            a.av = b.av;
+            a.ai = b.ai;
+        }
+    }
+}
+
+template <bool ARGMAX>
+__device__ __forceinline__ OnlineState shfl_xor_state(const OnlineState& st, int off) {
+    OnlineState o;
+    o.m = __shfl_xor_sync(0xffffffffu, st.m, off);
+    o.s = __shfl_xor_sync(0xffffffffu, st.s, off);
+    o.t = __shfl_xor_sync(0xffffffffu, st.t, off);
+    o.k = __shfl_xor_sync(0xffffffffu, st.k, off);
+    if constexpr (ARGMAX) {
+        o.av = __shfl_xor_sync(0xffffffffu, st.av, off);
+        o.ai = __shfl_xor_sync(0xffffffffu, st.ai, off);
+    } else {
+        o.av = 0.f;
+        o.ai = -1;
+    }
+    return o;
+}
+
+// Butterfly over groups of G lanes (G a power of two <= 32). Every lane of the
+// warp must call it. Addition and multiplication commute exactly, so every
+// lane of a group ends with the same bits.
+template <int G, bool ARGMAX>
+__device__ __forceinline__ void group_reduce(OnlineState& st) {
+#pragma unroll
+    for (int off = G / 2; off >= 1; off >>= 1) {
+        OnlineState o = shfl_xor_state<ARGMAX>(st, off);
+        merge<ARGMAX>(st, o);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Targets.
+__device__ __forceinline__ int64_t load_target(const void* y, int tdt, int64_t off) {
+    return tdt == 0 ? (int64_t)(reinterpret_cast<const int32_t*>(y)[off])
+                    : reinterpret_cast<const int64_t*>(y)[off];
+}
+
+// ---------------------------------------------------------------------------
+// Finalisation of one row from its complete state.
+//   lse  = m + log s, written as a float pair (hi, lo) with hi + lo = m + L to
+//          about 48 bits (two-sum of m and L = log s);
+//   loss = L - (1-eps)(z_y - m) - eps t/V   (t = sum_j (z_j - m))
+// ignore_index rows: loss 0. Out-of-range targets: loss NaN and error bit 1.
+struct RowOut {
+    float* loss;
+    float* lse;
+    float* lse_lo;
+    int32_t* argmax;
+    unsigned int* err;
+};
+
+__device__ __forceinline__ void finalize_row(const OnlineState& st, float zy, int64_t y,
+                                             int64_t ignore, int64_t V, float eps,
+                                             const RowOut& o, int64_t r, bool write_argmax) {
+    const float L = logf(st.s);
+    const float hi = st.m + L;
+    float lo = 0.f;
+    if (isfinite(hi)) {
+        const float bv = hi - st.m;
+        const float av = hi - bv;
+        lo = (st.m - av) + (L - bv);
+    }
+    o.lse[r] = hi;
+    if (o.lse_lo) o.lse_lo[r] = lo;
+    float loss;
+    if (y == ignore) {
+        loss = 0.f;
+    } else if (y < 0 || y >= V) {
+        loss = __int_as_float(0x7fc00000);
+        atomicOr(o.err, 1u);
+    } else {
+        loss = L - (1.f - eps) * (zy - st.m);
+        if (eps != 0.f) loss -= eps * (st.t / (float)V);
+    }
+    o.loss[r] = loss;
+    if (write_argmax) o.argmax[r] = st.ai < 0 ? 0 : st.ai;
+}
+
+}  // namespace ceb

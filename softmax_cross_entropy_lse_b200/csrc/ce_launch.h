@@ -1,0 +1,77 @@
+// Internal launch interface between the C ABI (ce_api.cu) and the kernel
+// translation units. Not part of the public header.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ceb {
+
+// Two-level row addressing: row r starts at (r / inner) * s_outer +
+// (r % inner) * s_inner elements, column j a further j * s_col on.
+struct Layout {
+    int64_t inner, s_outer, s_inner, s_col;
+};
+
+// ---- row forward -------------------------------------------------------------
+struct FwdArgs {
+    const void* z;
+    int64_t N, V;
+    const void* y;
+    int tdt;
+    float eps;
+    int64_t ignore;
+    float* loss;
+    float* lse;
+    float* lse_lo;
+    int32_t* argmax;
+    unsigned int* err;
+    float4* part;           // split partials [splits][N]
+    int splits;
+    int vec_is_scalar;
+    int64_t vec_per_split;  // in units of the kernel's vector width
+    Layout lz, ly;
+};
+
+struct FwdPlan {
+    enum Kind { kPacked = 0, kCta = 1 } kind;
+    int vec;        // 1 (scalar path) or the 16-byte vector width of the dtype
+    int G, U;       // packed: lanes per row, vectors per lane per step
+    int grid;
+    int merge_grid;
+    int splits;
+    int64_t vec_per_split;
+};
+
+cudaError_t launch_forward(const FwdPlan& p, const FwdArgs& a, int dtype, cudaStream_t s);
+int cta_threads_forward();
+
+// ---- row backward ------------------------------------------------------------
+struct BwdArgs {
+    const float* g;
+    int64_t g_stride;
+    const void* z;
+    int64_t N, V;
+    const void* y;
+    int tdt;
+    const float* lse;
+    const float* lse_lo;
+    float eps;
+    int64_t ignore;
+    void* dz;
+    unsigned int* err;
+    int64_t nchunks;
+    int64_t vec_per_chunk;
+    Layout lz, ly, ld;
+};
+
+struct BwdPlan {
+    int vec;
+    int G, U;
+    int grid;
+};
+
+cudaError_t launch_backward(const BwdPlan& p, const BwdArgs& a, int dt_in, int dt_out,
+                            cudaStream_t s);
+
+}  // namespace ceb
