@@ -1,0 +1,605 @@
+#!/usr/bin/env python
+"""Benchmark of the fused softmax cross-entropy hot path on B200.
+
+One step = one forward and one backward pass over one batch of synthetic,
+seeded input already resident in HBM (the row path: online log-sum-exp
+forward, then the VJP from the saved lse; the fused-linear path: forward and
+backward of Z = H W^T without storing Z). Default workload: 1,048,576 rows x
+128 classes, fp32 logits ~N(0,1), 10% of targets at ignore_index=-100,
+label smoothing 0.1.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2]
+    python bench.py --impl reference ...   (the float64 CPU oracle, timed)
+
+Prints one JSON line (rank 0). For N > 1 it is launched with torchrun, one
+rank per GPU; every rank processes its own batch (rows are independent, no
+data-path collective), the device time is the max over ranks and the value
+is the bytes of all ranks over that time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from softmax_cross_entropy_lse_b200 import workloads as wl  # noqa: E402
+
+METRIC = "CE fwd and fwd+bwd GB/s and rows/s vs HBM roofline; fused-linear TFLOP/s"
+
+# The pages' own numbers (Apple M5 Pro, MLX PR #4776 Benchmarks table, fix
+# column): forward + backward milliseconds for the same shape and dtype.
+# Another machine's numbers: context, not the target.
+PAGE_FWD_BWD_MS = {"c2": 6.364, "c3a": 6.073, "c3b": 7.263}
+
+ROW_WORKLOADS = {
+    "c1": dict(desc="4096 x 1024 fp32 rows ~N(0,1), uniform targets", dt="f32", eps=0.0),
+    "c2": dict(desc="1,048,576 x 128 fp32 rows ~N(0,1), 10% ignore_index=-100, label smoothing 0.1",
+               dt="f32", eps=wl.C2_EPS),
+    "c3a": dict(desc="8192 x 32000 bf16 rows ~N(0, std 2), bf16 dlogits", dt="bf16", eps=0.0),
+    "c3b": dict(desc="2048 x 151,936 bf16 rows ~N(0, std 2), bf16 dlogits", dt="bf16", eps=0.0),
+    "c4a": dict(desc="view x[:, :-1] of a (10, 119, 151,936) fp32 tensor vs t[:, 1:]", dt="f32",
+                eps=0.0),
+    "c4b": dict(desc="(2^27 + 2^20) x 8 fp32 rows ~N(0,1)", dt="f32", eps=0.0),
+}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), \
+            d.get("bf16_tflops_sustained", 1400.0), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "softmax_cross_entropy_lse_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("bytes_per_launch")
+
+
+# -- clocks during the timed region ---------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = f"/tmp/ce_bench_clocks_{os.getpid()}.csv"
+
+    def __enter__(self):
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.remove(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": float(np.median([r[0] for r in loaded])),
+                "sm_max_mhz": float(max(r[1] for r in rows)), "reasons": reasons,
+                "samples": len(rows), "power_w_max": float(max(r[2] for r in rows))}
+
+
+# -- distributed plumbing ---------------------------------------------------------------
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        pg = dist
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local, pg
+
+
+def sync_ranks(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+def max_over_ranks(pg, x: float) -> float:
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+# -- row workloads ------------------------------------------------------------------------
+def make_rows(workload: str, seed: int):
+    """Host arrays: (logits storage, float32 values, targets, layout kind)."""
+    if workload == "c4a":
+        x, t = wl.c4a(seed)
+        return x, x, t, "view"
+    if workload == "c4b":
+        n = (wl.C4B_ROWS + wl.C4B_CHUNK - 1) // wl.C4B_CHUNK
+        chunks = [wl.c4b_chunk(k, seed) for k in range(n)]
+        z = np.concatenate([c[0] for c in chunks])
+        y = np.concatenate([c[1] for c in chunks])
+        return z, z, y, "plain"
+    gen = {"c1": wl.c1, "c2": wl.c2, "c3a": wl.c3a, "c3b": wl.c3b}.get(workload)
+    if gen is None:
+        raise SystemExit(f"unknown workload {workload}")
+    z, z32, y = gen(seed)
+    return z, z32, y, "plain"
+
+
+def bench_rows(args, rank, world, pg):
+    import torch
+    import softmax_cross_entropy_lse_b200 as ce
+    spec = ROW_WORKLOADS[args.workload]
+    dt, eps = spec["dt"], spec["eps"]
+    z, z32, y, kind = make_rows(args.workload, seed=rank)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if dt == "bf16":
+        z_h = torch.from_numpy(np.ascontiguousarray(z).view(np.int16)).view(torch.bfloat16)
+    else:
+        z_h = torch.from_numpy(np.ascontiguousarray(z))
+    y_h = torch.from_numpy(np.ascontiguousarray(y))
+    z_d, y_d = z_h.to(dev), y_h.to(dev)
+
+    def views(zd, yd):
+        return (zd[:, :-1], yd[:, 1:]) if kind == "view" else (zd, yd)
+
+    zv, yv = views(z_d, y_d)
+    N = zv.numel() // zv.shape[-1]
+    V = zv.shape[-1]
+    esz = zv.element_size()
+    yflat = (y[:, 1:] if kind == "view" else y).reshape(-1)
+    n_valid = int((yflat != -100).sum())
+    g = torch.full((1,), 1.0 / max(n_valid, 1), dtype=torch.float32, device=dev)  # mean
+    dz = torch.empty(z_d.shape, dtype=z_d.dtype, device=dev)
+    dzv = views(dz, y_d)[0]
+    ws_bytes = ce.ce_workspace_size(N, V, zv.dtype)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # L2: a batch larger than L2 is read from HBM every step; a small batch
+    # rotates through enough copies that each is evicted before its reuse.
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    nbuf = 1
+    if z_d.numel() * esz < 2 * l2:
+        nbuf = int(np.ceil(3 * l2 / (z_d.numel() * esz)))
+    bufs = [(z_d, y_d, dz)] + [(z_d.clone(), y_d.clone(), torch.empty_like(dz))
+                               for _ in range(nbuf - 1)]
+
+    def step(i, ev=None):
+        zb, yb, db = bufs[i % nbuf]
+        zvb, yvb = views(zb, yb)
+        dvb = views(db, yb)[0]
+        if ev is not None:
+            ev[0].record(stream)
+        r = ce.ce_forward(zvb, yvb, eps, -100, workspace=ws)
+        if ev is not None:
+            ev[1].record(stream)
+        ce.ce_backward(g, zvb, yvb, r.lse, r.lse_lo, eps, -100, dlogits=dvb)
+        if ev is not None:
+            ev[2].record(stream)
+        return r
+
+    fwd_bytes = N * V * esz + 12 * N
+    bwd_bytes = 2 * N * V * esz + 12 * N
+    step_bytes = fwd_bytes + bwd_bytes
+    launches_per_step = (2 if ws_bytes > 0 else 1) + 1
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        sync_ranks(pg)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(i, evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        sync_ranks(pg)
+    ms = max_over_ranks(pg, t0.elapsed_time(t1))
+    fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+
+    # end to end through the public API with host buffers: pinned host inputs
+    # copied in, forward + backward, the per-row loss copied out, every step
+    z_pin = z_h.pin_memory()
+    y_pin = y_h.pin_memory()
+    loss_h = torch.empty(N, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        z_d.copy_(z_pin, non_blocking=True)
+        y_d.copy_(y_pin, non_blocking=True)
+        zv2, yv2 = views(z_d, y_d)
+        r = ce.ce_forward(zv2, yv2, eps, -100, workspace=ws)
+        ce.ce_backward(g, zv2, yv2, r.lse, r.lse_lo, eps, -100, dlogits=dzv)
+        loss_h.copy_(r.loss, non_blocking=True)
+
+    e2e_steps = max(2, min(args.steps, 10))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    sync_ranks(pg)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(pg, a.elapsed_time(b)) / e2e_steps
+    h2d = z_h.numel() * z_h.element_size() + y_h.numel() * y_h.element_size()
+    d2h = 4 * N
+
+    peak_hbm, _, _, peak_src = load_peaks()
+    dom, dom_ms, dom_bytes = ("backward", bwd_ms, bwd_bytes) if bwd_ms >= fwd_ms else \
+        ("forward", fwd_ms, fwd_bytes)
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    value = world * step_bytes * args.steps / (ms * 1e-3) / 1e9
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32" if dt == "f32" else "bf16", "data": "synthetic",
+        "rows_per_s": round(world * N * args.steps / (ms * 1e-3), 1),
+        "fwd_GBs": round(fwd_bytes / (fwd_ms * 1e-3) / 1e9, 2),
+        "fwd_rows_per_s": round(N / (fwd_ms * 1e-3), 1),
+        "bwd_GBs": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9, 2),
+        "config": {"workload": f"{args.workload}: {spec['desc']}; forward + backward",
+                   "rows": N, "classes": V, "label_smoothing": eps, "ignore_index": -100,
+                   "bytes_per_step": step_bytes,
+                   "l2": ("inputs larger than L2" if nbuf == 1 else
+                          f"{nbuf} rotating input buffers (total larger than L2)"),
+                   "parallelism": f"rows sharded, {world} independent replica(s), no collective"},
+        "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 2),
+                     "peak": peak_hbm, "unit": "GB/s", "frac": round(achieved / peak_hbm, 4),
+                     "traffic": recorded_traffic(args.workload, dom),
+                     "peak_source": peak_src, "algorithmic_bytes_per_launch": dom_bytes},
+    }
+    if args.workload in PAGE_FWD_BWD_MS:
+        page_gbs = step_bytes / (PAGE_FWD_BWD_MS[args.workload] * 1e-3) / 1e9
+        out["vs_baseline"] = round(value / page_gbs, 2)
+    clocks = clk.summary()
+    if clocks:
+        out["clocks"] = clocks
+    return out, (z32, y, eps, kind)
+
+
+# -- fused-linear workload -------------------------------------------------------------------
+def bench_linear(args, rank, world, pg):
+    import torch
+    import softmax_cross_entropy_lse_b200 as ce
+    N, V, D = 8192, 151936, 4096
+    hb, hf, wb, wf, y = wl.c5(seed=rank)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    H_h = torch.from_numpy(hb.view(np.int16)).view(torch.bfloat16)
+    W_h = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16)
+    y_h = torch.from_numpy(y)
+    H, W, yd = H_h.to(dev), W_h.to(dev), y_h.to(dev)
+    g = torch.full((1,), 1.0 / N, dtype=torch.float32, device=dev)
+    L = ce.lib()
+    ws_f = torch.empty(max(L.linear_ce_workspace_size(N, V, D, 0), 16), dtype=torch.uint8,
+                       device=dev)
+    ws_b = torch.empty(max(L.linear_ce_backward_workspace_size(N, V, D, 0), 16),
+                       dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        loss, lse = ce.linear_ce_forward(H, W, yd, workspace=ws_f)
+        if ev is not None:
+            ev[1].record(stream)
+        ce.linear_ce_backward(g, H, W, yd, lse, workspace=ws_b)
+        if ev is not None:
+            ev[2].record(stream)
+
+    fwd_flop = 2.0 * N * V * D
+    bwd_flop = 3 * fwd_flop
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        sync_ranks(pg)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        sync_ranks(pg)
+    ms = max_over_ranks(pg, t0.elapsed_time(t1))
+    fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    _, peak_burst, peak_sust, src = load_peaks()
+    step_flop = fwd_flop + bwd_flop
+    value = world * step_flop * args.steps / (ms * 1e-3) / 1e12
+    # e2e: H, W and targets copied in from pinned host memory each step, loss out
+    Hp, Wp, yp = H_h.pin_memory(), W_h.pin_memory(), y_h.pin_memory()
+    loss_h = torch.empty(N, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        H.copy_(Hp, non_blocking=True)
+        W.copy_(Wp, non_blocking=True)
+        yd.copy_(yp, non_blocking=True)
+        loss, lse = ce.linear_ce_forward(H, W, yd, workspace=ws_f)
+        ce.linear_ce_backward(g, H, W, yd, lse, workspace=ws_b)
+        loss_h.copy_(loss, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    sync_ranks(pg)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(2):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(pg, a.elapsed_time(b)) / 2
+    dom, dom_ms, dom_flop = ("backward", bwd_ms, bwd_flop) if bwd_ms >= fwd_ms else \
+        ("forward", fwd_ms, fwd_flop)
+    achieved = dom_flop / (dom_ms * 1e-3) / 1e12
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "fwd_tflops": round(fwd_flop / (fwd_ms * 1e-3) / 1e12, 2), "fwd_ms": round(fwd_ms, 4),
+        "bwd_ms": round(bwd_ms, 4),
+        "config": {"workload": "c5: fused linear CE, H (8192, 4096) bf16 ~N(0,1), W (151,936, 4096) "
+                               "bf16 ~N(0, std 0.02), forward + backward (logits recomputed)",
+                   "N": N, "V": V, "D": D, "flop_per_step": step_flop,
+                   "l2": "operands larger than L2 (W is 1.24 GB)",
+                   "parallelism": f"rows sharded, {world} independent replica(s), no collective"},
+        "e2e": {"value": round(world * step_flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": (N * D + V * D) * 2 + 4 * N, "d2h_bytes_per_step": 4 * N},
+        "gpu_launches": None,
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2),
+                     "peak": peak_sust, "unit": "TFLOP/s", "frac": round(achieved / peak_sust, 4),
+                     "traffic": recorded_traffic("c5", dom), "peak_source": src + " (sustained)"},
+    }
+    clocks = clk.summary()
+    if clocks:
+        out["clocks"] = clocks
+    return out, None
+
+
+# -- CPU oracle ---------------------------------------------------------------------------------
+class OracleRows:
+    """The float64 oracle (forward + backward) over whole rows of a row workload."""
+
+    def __init__(self, workload, host=None):
+        import oracle
+        self.orc = oracle.get()
+        spec = ROW_WORKLOADS[workload]
+        self.eps = spec["eps"]
+        self.esz = 4 if spec["dt"] == "f32" else 2
+        if host is None:
+            _, z32, y, kind = make_rows(workload, 0)
+        else:
+            z32, y, kind = host[0], host[1], host[3]
+        if kind == "view":
+            V = z32.shape[-1]
+            z32 = z32[:, :-1].reshape(-1, V)
+            y = y[:, 1:].reshape(-1)
+        self.z32, self.y = z32, y
+        self.N, self.V = z32.shape
+        self.bytes_per_row = 3 * self.V * self.esz + 24
+        self.cursor = 0
+
+    def run(self, rows: int) -> None:
+        done = 0
+        chunk = max(1, int(5e7 // self.V))
+        while done < rows:
+            lo = self.cursor % self.N
+            n = min(chunk, rows - done, self.N - lo)
+            zc = self.z32[lo:lo + n].astype(np.float64)
+            self.orc.ce_forward(zc, self.y[lo:lo + n], self.eps)
+            self.orc.ce_backward(zc, self.y[lo:lo + n], 1.0, self.eps)
+            self.cursor += n
+            done += n
+
+    def rows_for(self, seconds: float) -> int:
+        probe = min(self.N, max(1, int(2e6 // self.V)))
+        t = time.perf_counter()
+        self.run(probe)
+        per_row = max((time.perf_counter() - t) / probe, 1e-9)
+        self.cursor = 0
+        return int(max(1, seconds / per_row))
+
+
+class OracleLinear:
+    """The float64 oracle on whole rows of the fused-linear workload (loss,
+    lse and the dH row of each sampled row)."""
+
+    def __init__(self):
+        import oracle
+        self.orc = oracle.get()
+        self.N, self.V, self.D = 8192, 151936, 4096
+        _, self.hf, _, self.wf, self.y = wl.c5(seed=0)
+        self.cursor = 0
+        self.flop_per_row = 4.0 * self.V * self.D
+
+    def run(self, rows: int) -> None:
+        r = (self.cursor + np.arange(rows)) % self.N
+        self.orc.linear_ce_forward_rows(self.hf, self.wf, self.y, rows=r)
+        self.orc.linear_ce_dh_rows(self.hf, self.wf, self.y, 1.0 / self.N, rows=r)
+        self.cursor += rows
+
+    def rows_for(self, seconds: float) -> int:
+        n = max(1, self.orc.num_threads())
+        t = time.perf_counter()
+        self.run(n)
+        per_row = (time.perf_counter() - t) / n
+        self.cursor = 0
+        return int(max(n, (seconds / per_row) // n * n))
+
+
+def oracle_baseline(workload, seconds: float, host=None):
+    """(value, unit, cores, sample) of the oracle timed for about `seconds`."""
+    if workload == "c5":
+        o = OracleLinear()
+        rows = o.rows_for(seconds)
+        t = time.perf_counter()
+        o.run(rows)
+        dt = time.perf_counter() - t
+        return (rows * o.flop_per_row / dt / 1e12, "TFLOP/s", o.orc.num_threads(),
+                f"{rows} of 8192 rows of c5 (loss, lse and dH rows), {dt:.1f} s")
+    o = OracleRows(workload, host)
+    rows = min(o.rows_for(seconds), 50 * o.N)
+    t = time.perf_counter()
+    o.run(rows)
+    dt = time.perf_counter() - t
+    return (rows * o.bytes_per_row / dt / 1e9, "GB/s", o.orc.num_threads(),
+            f"{rows} rows of {workload} ({rows / o.N:.3g} batches), forward + backward, {dt:.1f} s")
+
+
+def run_reference(args):
+    """The reference arm: the float64 oracle, as it stands, on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    if args.workload == "c5":
+        o = OracleLinear()
+        unit, per_row = "TFLOP/s", o.flop_per_row / 1e12
+    else:
+        o = OracleRows(args.workload)
+        unit, per_row = "GB/s", o.bytes_per_row / 1e9
+    # each step a bounded sample, so the whole run stays within about two minutes
+    step_s = min(2.0, 120.0 / (args.steps + args.warmup))
+    rows = o.rows_for(step_s)
+    for _ in range(args.warmup):
+        o.run(rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        o.run(rows)
+    wall = time.perf_counter() - t0
+    value = rows * args.steps * per_row / wall
+    cores = o.orc.num_threads()
+    sample = f"{rows} rows of {args.workload} per step, forward + backward in float64"
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": unit,
+            "n_gpus": int(os.environ.get("WORLD_SIZE", args.gpus)), "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(wall * 1e3 / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "sample_rows_per_step": rows},
+            "gpu_launches": 0,
+            "cpu_baseline": {"value": round(value, 4), "unit": unit, "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="c2", choices=sorted(ROW_WORKLOADS) + ["c5"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    rank, world, local, pg = dist_setup(args.gpus)
+    if args.workload == "c5":
+        out, host = bench_linear(args, rank, world, pg)
+    else:
+        out, host = bench_rows(args, rank, world, pg)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, unit, cores, sample = oracle_baseline(args.workload, 12.0, host)
+        out["cpu_baseline"] = {"value": round(v, 4), "unit": unit, "cores": cores,
+                               "kind": "oracle", "sample": sample}
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

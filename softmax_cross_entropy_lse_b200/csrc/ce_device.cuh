@@ -223,6 +223,62 @@ __device__ __forceinline__ void fold(OnlineState& st, const float* v, int col0, 
     }
 }
 
+// Folds U vectors of VEC values, of which only those with ok[u] set are
+// valid (MASKED) or all (not MASKED): one max, one rescale, one exponential
+// per valid element.
+template <int U, int VEC, bool MASKED>
+__device__ __forceinline__ void fold_vecs(OnlineState& st, const float (&v)[U][VEC],
+                                          const bool (&ok)[U]) {
+    float cm = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        if (MASKED && !ok[u]) continue;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) cm = fmaxf(cm, v[u][e]);
+    }
+    rescale_to(st, fmaxf(st.m, cm));
+    const float ms = (st.m == -INFINITY) ? 0.f : st.m;
+    float sa = 0.f, ta = 0.f;
+    int n = 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        if (MASKED && !ok[u]) continue;
+        float su = 0.f, tu = 0.f;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            const float d = v[u][e] - ms;
+            su += ex2(d * kLog2e);
+            tu += d;
+        }
+        sa += su;
+        ta += tu;
+        n += VEC;
+    }
+    st.s += sa;
+    st.t += ta;
+    st.k += n;
+}
+
+// Argmax over U vectors whose first columns are col0[u], in increasing
+// column order per thread (a strict comparison keeps the first of equals).
+template <int U, int VEC, bool MASKED>
+__device__ __forceinline__ void argmax_vecs(OnlineState& st, const float (&v)[U][VEC],
+                                            const bool (&ok)[U], const int (&col0)[U]) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        if (MASKED && !ok[u]) continue;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            const float x = v[u][e];
+            const bool take = (st.ai < 0) | (x > st.av) | ((x != x) & (st.av == st.av));
+            if (take) {
+                st.av = x;
+                st.ai = col0[u] + e;
+            }
+        }
+    }
+}
+
 template <bool ARGMAX>
 __device__ __forceinline__ void merge(OnlineState& a, const OnlineState& b) {
     const float M = fmaxf(a.m, b.m);

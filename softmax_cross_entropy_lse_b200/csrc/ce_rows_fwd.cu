@@ -46,38 +46,21 @@ __global__ void __launch_bounds__(256) k_fwd_packed(FwdArgs a) {
             for (int64_t vb = 0; vb < nvec; vb += (int64_t)G * U) {
                 float v[U][VEC];
                 bool ok[U];
+                int c0[U];
+                const bool full = vb + (int64_t)G * U <= nvec;
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     const int64_t vi = vb + u * G + gl;
-                    ok[u] = vi < nvec;
+                    ok[u] = full || vi < nvec;
+                    c0[u] = (int)(vi * VEC);
                     if (ok[u]) load_vec<T, VEC>(row, vi * VEC, a.lz.s_col, v[u]);
                 }
-                if (vb + (int64_t)G * U <= nvec) {
-                    // every vector of this step is in range: one fold of U*VEC values
-                    fold<U * VEC, false>(st, &v[0][0], 0, 0);
+                if (full) {
+                    fold_vecs<U, VEC, false>(st, v, ok);
+                    if constexpr (ARGMAX) argmax_vecs<U, VEC, false>(st, v, ok, c0);
                 } else {
-#pragma unroll
-                    for (int u = 0; u < U; ++u)
-                        if (ok[u]) fold<VEC, false>(st, v[u], 0, 0);
-                }
-                if constexpr (ARGMAX) {
-                    // columns of one lane are visited in increasing order, so a
-                    // strict comparison keeps the first of equal values
-#pragma unroll
-                    for (int u = 0; u < U; ++u) {
-                        if (!ok[u]) continue;
-                        const int c0 = (int)((vb + u * G + gl) * VEC);
-#pragma unroll
-                        for (int q = 0; q < VEC; ++q) {
-                            const float x = v[u][q];
-                            const bool take =
-                                (st.ai < 0) | (x > st.av) | ((x != x) & (st.av == st.av));
-                            if (take) {
-                                st.av = x;
-                                st.ai = c0 + q;
-                            }
-                        }
-                    }
+                    fold_vecs<U, VEC, true>(st, v, ok);
+                    if constexpr (ARGMAX) argmax_vecs<U, VEC, true>(st, v, ok, c0);
                 }
             }
             // ragged tail: the last V % VEC columns, one per lane
@@ -133,33 +116,27 @@ __global__ void __launch_bounds__(kCtaThreads, kCtaMinBlocks) k_fwd_cta(FwdArgs 
         }
 
         OnlineState st = empty_state();
-        int64_t vb = v0;
-        for (; vb + (int64_t)kCtaThreads * U <= v1; vb += (int64_t)kCtaThreads * U) {
+        // every step issues U 16-byte loads per thread before using any of
+        // them; only the last step of a unit needs predicates
+        for (int64_t vb = v0; vb < v1; vb += (int64_t)kCtaThreads * U) {
             float v[U][VEC];
+            bool ok[U];
+            int c0[U];
+            const bool full = vb + (int64_t)kCtaThreads * U <= v1;
 #pragma unroll
-            for (int q = 0; q < U; ++q)
-                load_vec<T, VEC>(row, (vb + q * kCtaThreads + tid) * VEC, a.lz.s_col, v[q]);
-            fold<U * VEC, false>(st, &v[0][0], 0, 0);
-            if constexpr (ARGMAX) {
-#pragma unroll
-                for (int q = 0; q < U; ++q) {
-                    const int c0 = (int)((vb + q * kCtaThreads + tid) * VEC);
-#pragma unroll
-                    for (int e = 0; e < VEC; ++e) {
-                        const float x = v[q][e];
-                        const bool take = (st.ai < 0) | (x > st.av) | ((x != x) & (st.av == st.av));
-                        if (take) {
-                            st.av = x;
-                            st.ai = c0 + e;
-                        }
-                    }
-                }
+            for (int q = 0; q < U; ++q) {
+                const int64_t vi = vb + q * kCtaThreads + tid;
+                ok[q] = full || vi < v1;
+                c0[q] = (int)(vi * VEC);
+                if (ok[q]) load_vec<T, VEC>(row, vi * VEC, a.lz.s_col, v[q]);
             }
-        }
-        for (int64_t vi = vb + tid; vi < v1; vi += kCtaThreads) {
-            float v[VEC];
-            load_vec<T, VEC>(row, vi * VEC, a.lz.s_col, v);
-            fold<VEC, ARGMAX>(st, v, (int)(vi * VEC), 1);
+            if (full) {
+                fold_vecs<U, VEC, false>(st, v, ok);
+                if constexpr (ARGMAX) argmax_vecs<U, VEC, false>(st, v, ok, c0);
+            } else {
+                fold_vecs<U, VEC, true>(st, v, ok);
+                if constexpr (ARGMAX) argmax_vecs<U, VEC, true>(st, v, ok, c0);
+            }
         }
         if (sp == a.splits - 1) {
             for (int q = tid; q < tail; q += kCtaThreads) {
