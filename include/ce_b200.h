@@ -7,9 +7,9 @@
  *
  * Ownership. The caller owns every buffer, the workspace and the stream. The
  * library allocates no device memory per call and writes nothing but the
- * outputs named in each call and the workspace handed to it. The one piece
- * of library-owned device state is a per-device error word (see
- * ce_get_error).
+ * outputs named in each call and the workspace handed to it. Library-owned
+ * device state: a per-device error word (see ce_get_error) and the scratch
+ * array of ce_forward_noalloc.
  *
  * Completion. Calls are asynchronous: they validate their arguments on the
  * host, enqueue kernels on `cuda_stream` and return. Every output element is
@@ -181,6 +181,39 @@ ce_status linear_ce_backward(const float* grad_out, int64_t grad_stride,
                              float label_smoothing, int64_t ignore_index,
                              void* dH, ce_dtype dH_dt, void* dW, ce_dtype dW_dt,
                              void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* ------------------------------------------------------------------------ *
+ * Forward without a caller-provided workspace.
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot allocate device memory or pass a workspace: code running while a
+ * stream is being captured into a CUDA graph (allocation is refused there),
+ * plugin hosts that own all device memory through their own pool, and C
+ * callers without an allocator.
+ *
+ * Same arguments, results and errors as ce_forward, without workspace and
+ * ws_bytes. The scratch for the vocabulary split lives in a library-owned
+ * array of CE_NOALLOC_SCRATCH_BYTES (64 KiB) in device memory, one per device
+ * that loads the library, held until the process exits. On a 148-SM B200
+ * that holds the split partials of every shape whose rows are at most
+ * 128 KB (32768 fp32 or 65536 bf16 classes) and of longer rows for up to 32
+ * rows (and many larger counts); a shape whose ce_workspace_size exceeds it
+ * returns CE_EWORKSPACE and enqueues nothing.
+ * The call allocates nothing. The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress, with that device current) and caches
+ * it; make that first call before any stream capture begins. All calls on a
+ * device share the one array and it keeps the last call's partial states:
+ * calls whose kernels can overlap on the GPU (different streams, no ordering
+ * between them) race on it and must be serialised by the caller. Nothing in
+ * the array needs to start at zero: each call writes every slot it reads.
+ * ------------------------------------------------------------------------ */
+#define CE_NOALLOC_SCRATCH_BYTES ((size_t)64 << 10)
+
+ce_status ce_forward_noalloc(const void* logits, ce_dtype dt, ce_layout lg,
+                             int64_t N, int64_t V,
+                             const void* targets, ce_index_dtype tdt, ce_layout tg,
+                             float label_smoothing, int64_t ignore_index,
+                             float* loss, float* lse, float* lse_lo, int32_t* argmax,
+                             void* cuda_stream);
 
 /* ------------------------------------------------------------------------ */
 

@@ -25,7 +25,8 @@ STATUS = {0: "CE_OK", 1: "CE_EINVAL", 2: "CE_EALIAS", 3: "CE_EWORKSPACE", 4: "CE
           5: "CE_ETARGET", 6: "CE_ENOTSUP"}
 EXPORTED = ["ce_workspace_size", "ce_forward", "ce_backward", "linear_ce_workspace_size",
             "linear_ce_forward", "linear_ce_backward_workspace_size", "linear_ce_backward",
-            "ce_get_error", "ce_status_string"]
+            "ce_get_error", "ce_status_string", "ce_forward_noalloc"]
+NOALLOC_SCRATCH_BYTES = 64 << 10
 
 
 class ce_layout(ctypes.Structure):
@@ -70,6 +71,9 @@ def lib() -> ctypes.CDLL:
         L.linear_ce_backward.argtypes = [vp, i64, vp, i64, vp, i64, vp, ctypes.c_int, vp, i64, i64,
                                          i64, f32, i64, vp, ctypes.c_int, vp, ctypes.c_int, vp, sz, vp]
         L.linear_ce_backward.restype = ctypes.c_int
+        L.ce_forward_noalloc.argtypes = [vp, ctypes.c_int, ce_layout, i64, i64, vp, ctypes.c_int,
+                                         ce_layout, f32, i64, vp, vp, vp, vp, vp]
+        L.ce_forward_noalloc.restype = ctypes.c_int
         L.ce_get_error.argtypes = [vp]
         L.ce_get_error.restype = ctypes.c_int
         L.ce_status_string.argtypes = [ctypes.c_int]
