@@ -1,25 +1,738 @@
-// Fused-linear cross-entropy (Z = H W^T never stored). Placeholder entry
-// points until the tensor-core kernels land.
+// Fused-linear cross-entropy on sm_100a tensor cores.
+//
+// Source: Ineshin, "A fused linear cross-entropy forward kernel for Apple
+// GPUs", section 1: with H (N x D) and W (V x D), the logits Z = H W^T are
+// produced tile by tile, each vocabulary tile is folded into the running
+// (max, scaled sum) state of every row, the target logit is captured when its
+// tile passes, and the (N, V) matrix never exists. The backward regenerates
+// the logits tile by tile from the saved log-sum-exp.
+//
+// Design for B200 (not the page's Metal kernel):
+//  * one persistent GEMM engine, 128 x 256 output tiles, K in 64-element
+//    (128-byte) steps: a TMA producer warp fills a 4-stage shared-memory ring,
+//    one thread issues tcgen05.mma into a double-buffered f32 accumulator in
+//    tensor memory (2 x 256 columns), and four epilogue warps read the
+//    accumulator with tcgen05.ld, one TMEM lane (= one output row) per thread;
+//  * forward epilogue: the online log-sum-exp of each row over a unit of
+//    consecutive vocabulary tiles, kept in registers, then a partial state
+//    per (unit, row) merged in unit order by a second launch;
+//  * backward: for each vocabulary chunk, GEMM 1 recomputes Z_c = H W_c^T and
+//    its epilogue writes G_c = g (softmax - (1-eps) onehot - eps/V) in bf16
+//    (row-major and transposed); GEMM 2 forms dW_c = G_c^T H; GEMM 3 adds
+//    G_c W_c into a float dH accumulator. Each dW row belongs to one chunk,
+//    so dW needs no accumulation across chunks.
+// Every pipeline wait is bounded in time; on expiry the CTA raises an error
+// bit, drains its own copies and MMAs, frees its tensor memory and returns.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "ce_b200.h"
+#include "ce_device.cuh"
 #include "ce_linear.h"
+#include "ce_sm100.cuh"
+
+namespace ceb {
+using namespace sm100;
+
+constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4;
+constexpr uint32_t kABytes = kBM * kBK * 2;
+constexpr uint32_t kBBytes = kBN * kBK * 2;
+constexpr uint32_t kStageBytes = kABytes + kBBytes;
+constexpr int kGemmThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
+constexpr uint32_t kTmemCols = 2 * kBN;
+constexpr size_t kGemmSmem = 1024 + (size_t)kStages * kStageBytes + 256;
+constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN);
+constexpr unsigned kErrTimeout = 2u;
+
+enum EpiKind { kEpiCeFwd = 0, kEpiCeGrad = 1, kEpiStore = 2, kEpiAccum = 3 };
+
+struct GemmArgs {
+    int M, Nn, K;              // output rows, output columns, reduction length
+    int n_mb, n_nb, nkb;       // tile counts
+    int tiles_per_unit;        // consecutive column tiles handled as one unit
+    int n_units_n;             // ceil(n_nb / tiles_per_unit)
+    int64_t units;             // n_mb * n_units_n
+    int kA0, kB0;              // K origin of A and B in their tensor maps
+    unsigned int* err;
+    // cross-entropy epilogues
+    const void* y;
+    int tdt;
+    int64_t V;
+    float eps;
+    int64_t ignore;
+    int64_t col_base;          // vocabulary index of output column 0
+    float4* part;              // forward partials [n_units_n][M]
+    const float* g;
+    int64_t g_stride;
+    const float* lse;
+    __nv_bfloat16* G;          // gradient chunk, row-major, ld = ldG
+    int64_t ldG;
+    __nv_bfloat16* GT;         // its transpose, ld = ldGT
+    int64_t ldGT;
+    // store / accumulate epilogues
+    void* C;                   // output rows start here
+    int64_t ldc;
+    int c_f32;
+    float* acc;                // float accumulator (may equal C when c_f32)
+    int64_t ld_acc;
+    int acc_first, acc_last;
+};
+
+// ---------------------------------------------------------------------------
+// Epilogue helpers.
+
+// Folds the first nv of 32 values (nv < 32 only in a ragged last tile).
+__device__ __forceinline__ void fold_prefix(OnlineState& st, const float (&v)[32], int nv) {
+    float cm = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+        if (j < nv) cm = fmaxf(cm, v[j]);
+    rescale_to(st, fmaxf(st.m, cm));
+    const float ms = (st.m == -INFINITY) ? 0.f : st.m;
+    float sa = 0.f, ta = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        if (j < nv) {
+            const float d = v[j] - ms;
+            sa += ex2(d * kLog2e);
+            ta += d;
+        }
+    }
+    st.s += sa;
+    st.t += ta;
+    st.k += nv;
+}
+
+__device__ __forceinline__ void store_row32(void* base, int64_t ld, int64_t row, int64_t col,
+                                            const float (&v)[32], int f32, int ncols) {
+    if (f32) {
+        float* p = reinterpret_cast<float*>(base) + row * ld + col;
+        if (ncols == 32) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                reinterpret_cast<float4*>(p)[q] =
+                    make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (j < ncols) p[j] = v[j];
+        }
+    } else {
+        __nv_bfloat16* p = reinterpret_cast<__nv_bfloat16*>(base) + row * ld + col;
+        if (ncols == 32) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint4 w;
+                w.x = pack2((__nv_bfloat16*)nullptr, v[8 * q], v[8 * q + 1]);
+                w.y = pack2((__nv_bfloat16*)nullptr, v[8 * q + 2], v[8 * q + 3]);
+                w.z = pack2((__nv_bfloat16*)nullptr, v[8 * q + 4], v[8 * q + 5]);
+                w.w = pack2((__nv_bfloat16*)nullptr, v[8 * q + 6], v[8 * q + 7]);
+                reinterpret_cast<uint4*>(p)[q] = w;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (j < ncols) p[j] = __float2bfloat16_rn(v[j]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// The persistent GEMM: C[M x Nn] = A[M x K] * B[Nn x K]^T, bf16 K-major
+// operands through TMA tensor maps, f32 accumulation in tensor memory.
+template <int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+           const GemmArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kStages * kABytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (size_t)kStages * kStageBytes);
+    // barrier slots: full[kStages], empty[kStages], tfull[2], tempty[2], drain
+    const uint32_t bar0 = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+    auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * kStages + b); };
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 2 + b); };
+    const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kStages + 5);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 128);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch(&tmA);
+        tma_prefetch(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            uint32_t issued_mask = 0, last_ph = 0;  // per stage: has a load, its phase
+            bool ok = true;
+            for (int64_t u = blockIdx.x; u < a.units && ok; u += gridDim.x) {
+                const int mb = (int)(u % a.n_mb);
+                const int un = (int)(u / a.n_mb);
+                const int nb0 = un * a.tiles_per_unit;
+                const int nb1 = min(a.n_nb, nb0 + a.tiles_per_unit);
+                for (int nb = nb0; nb < nb1 && ok; ++nb) {
+                    for (int kb = 0; kb < a.nkb; ++kb) {
+                        if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_expect_tx(full_bar(s), kStageBytes);
+                        tma_load_2d(smem_u32(sA + s * kABytes), &tmA, full_bar(s),
+                                    a.kA0 + kb * kBK, mb * kBM);
+                        tma_load_2d(smem_u32(sB + s * kBBytes), &tmB, full_bar(s),
+                                    a.kB0 + kb * kBK, nb * kBN);
+                        issued_mask |= 1u << s;
+                        last_ph = (last_ph & ~(1u << s)) | (ph << s);
+                        if (++s == kStages) {
+                            s = 0;
+                            ph ^= 1u;
+                        }
+                    }
+                }
+            }
+            if (!ok) {
+                atomicOr(a.err, kErrTimeout);
+                // let every copy this thread started land before the CTA exits
+                volatile int never = 0;
+                for (int q = 0; q < kStages; ++q)
+                    if (issued_mask & (1u << q)) mbar_wait(full_bar(q), (last_ph >> q) & 1u, &never);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (one thread) ----------------
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0, it = 0;
+            bool ok = true;
+            for (int64_t u = blockIdx.x; u < a.units && ok; u += gridDim.x) {
+                const int un = (int)(u / a.n_mb);
+                const int nb0 = un * a.tiles_per_unit;
+                const int nb1 = min(a.n_nb, nb0 + a.tiles_per_unit);
+                for (int nb = nb0; nb < nb1 && ok; ++nb, ++it) {
+                    const uint32_t acc = it & 1u;
+                    if (!mbar_wait(tempty_bar(acc), ((it >> 1) & 1u) ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d = tmem_base + acc * kBN;
+                    for (int kb = 0; kb < a.nkb; ++kb) {
+                        if (!mbar_wait(full_bar(s), ph, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t a0 = smem_u32(sA + s * kABytes);
+                        const uint32_t b0 = smem_u32(sB + s * kBBytes);
+#pragma unroll
+                        for (int kk = 0; kk < kBK / 16; ++kk)
+                            umma_bf16(d, desc_kmajor_sw128(a0 + kk * 32),
+                                      desc_kmajor_sw128(b0 + kk * 32), kIdesc,
+                                      (kb | kk) != 0 ? 1u : 0u);
+                        umma_commit(empty_bar(s));
+                        if (++s == kStages) {
+                            s = 0;
+                            ph ^= 1u;
+                        }
+                    }
+                    if (ok) umma_commit(tfull_bar(acc));
+                }
+            }
+            if (!ok) atomicOr(a.err, kErrTimeout);
+            // every MMA this thread issued has completed once `drain` flips
+            umma_commit(drain_bar);
+            volatile int never = 0;
+            mbar_wait(drain_bar, 0, &never);
+        }
+    } else {
+        // ---------------- epilogue: warps 2..5, TMEM lane quadrant warp % 4 ----
+        const int q = warp & 3;
+        const int r_in_tile = 32 * q + lane;
+        const uint32_t lane_addr = (uint32_t)(32 * q) << 16;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int64_t u = blockIdx.x; u < a.units && ok; u += gridDim.x) {
+            const int mb = (int)(u % a.n_mb);
+            const int un = (int)(u / a.n_mb);
+            const int nb0 = un * a.tiles_per_unit;
+            const int nb1 = min(a.n_nb, nb0 + a.tiles_per_unit);
+            const int64_t m = (int64_t)mb * kBM + r_in_tile;
+            const bool row_ok = m < a.M;
+
+            // per-row state of the cross-entropy epilogues
+            OnlineState st = empty_state();
+            int64_t y = 0;
+            float zy = 0.f, gl = 0.f, lse = 0.f, c_eps = 0.f, c_tgt = 0.f;
+            bool live = false;
+            if constexpr (EPI == kEpiCeFwd || EPI == kEpiCeGrad) {
+                if (row_ok) y = load_target(a.y, a.tdt, m);
+            }
+            if constexpr (EPI == kEpiCeGrad) {
+                if (row_ok) {
+                    const bool bad = y != a.ignore && (y < 0 || y >= a.V);
+                    live = y != a.ignore && !bad;
+                    if (bad && a.col_base == 0) atomicOr(a.err, 1u);
+                    gl = a.g[m * a.g_stride];
+                    lse = a.lse[m];
+                    c_eps = gl * a.eps / (float)a.V;
+                    c_tgt = gl * (1.f - a.eps);
+                }
+            }
+
+            for (int nb = nb0; nb < nb1; ++nb, ++it) {
+                const uint32_t acc = it & 1u;
+                if (!mbar_wait(tfull_bar(acc), (it >> 1) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t t0 = tmem_base + lane_addr + acc * kBN;
+                const int64_t col0 = (int64_t)nb * kBN;  // output column of chunk 0
+                int valid = (int)min((int64_t)kBN, (int64_t)a.Nn - col0);
+#pragma unroll 1
+                for (int ch = 0; ch < kBN / 32; ++ch) {
+                    if (ch * 32 >= valid) break;
+                    uint32_t r[32];
+                    tmem_ld32(t0 + ch * 32, r);
+                    tmem_wait_ld();
+                    float v[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+                    const int nv = min(32, valid - ch * 32);
+                    const int64_t c = col0 + ch * 32;  // output column of v[0]
+                    if constexpr (EPI == kEpiCeFwd) {
+                        if (nv == 32)
+                            fold<32, false>(st, v, 0, 0);
+                        else
+                            fold_prefix(st, v, nv);
+                        const int64_t dy = y - (a.col_base + c);
+                        if (row_ok && dy >= 0 && dy < 32) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (j == dy) zy = v[j];
+                        }
+                    } else if constexpr (EPI == kEpiCeGrad) {
+                        // G = g (exp(z - lse) - eps/V) - g (1 - eps)[col = y]
+                        const int64_t dy = y - (a.col_base + c);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            float gv = 0.f;
+                            if (live && j < nv) {
+                                gv = fmaf(gl, ex2((v[j] - lse) * kLog2e), -c_eps);
+                                if (j == dy) gv -= c_tgt;
+                            }
+                            v[j] = gv;
+                        }
+                        if (row_ok) store_row32(a.G, a.ldG, m, c, v, 0, nv);
+                        // transposed copy: column j of this chunk is row c + j of
+                        // G^T; the 32 lanes write 32 consecutive rows' entries
+                        if (row_ok) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if (j < nv) a.GT[(c + j) * a.ldGT + m] = __float2bfloat16_rn(v[j]);
+                        }
+                    } else if constexpr (EPI == kEpiStore) {
+                        if (row_ok) store_row32(a.C, a.ldc, m, c, v, a.c_f32, nv);
+                    } else {  // kEpiAccum
+                        if (row_ok) {
+                            float* p = a.acc + m * a.ld_acc + c;
+                            if (!a.acc_first) {
+                                if (nv == 32) {
+#pragma unroll
+                                    for (int q4 = 0; q4 < 8; ++q4) {
+                                        const float4 o = reinterpret_cast<const float4*>(p)[q4];
+                                        v[4 * q4] += o.x;
+                                        v[4 * q4 + 1] += o.y;
+                                        v[4 * q4 + 2] += o.z;
+                                        v[4 * q4 + 3] += o.w;
+                                    }
+                                } else {
+#pragma unroll
+                                    for (int j = 0; j < 32; ++j)
+                                        if (j < nv) v[j] += p[j];
+                                }
+                            }
+                            if (a.acc_last)
+                                store_row32(a.C, a.ldc, m, c, v, a.c_f32, nv);
+                            else
+                                store_row32(a.acc, a.ld_acc, m, c, v, 1, nv);
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(tempty_bar(acc));
+            }
+            if constexpr (EPI == kEpiCeFwd) {
+                if (ok && row_ok) a.part[(int64_t)un * a.M + m] = make_float4(st.m, st.s, st.t, zy);
+            }
+        }
+        if (!ok) atomicOr(a.err, kErrTimeout);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// Merge of the forward partials, in unit order, one thread per row.
+__global__ void __launch_bounds__(256) k_linear_merge(const float4* part, int64_t N, int64_t V,
+                                                      int tile_cols_per_unit, int n_units,
+                                                      const void* y_ptr, int tdt, float eps,
+                                                      int64_t ignore, float* loss, float* lse,
+                                                      unsigned int* err) {
+    const RowOut out{loss, lse, nullptr, nullptr, err};
+    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < N;
+         r += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t y = load_target(y_ptr, tdt, r);
+        const int64_t uy = (y >= 0 && y < V) ? y / tile_cols_per_unit : -1;
+        OnlineState st = empty_state();
+        float zy = 0.f;
+        for (int un = 0; un < n_units; ++un) {
+            const float4 rec = part[(int64_t)un * N + r];
+            const int64_t c0 = (int64_t)un * tile_cols_per_unit;
+            const int64_t c1 = min(V, c0 + tile_cols_per_unit);
+            OnlineState o;
+            o.m = rec.x;
+            o.s = rec.y;
+            o.t = rec.z;
+            o.k = (int)(c1 - c0);
+            o.av = 0.f;
+            o.ai = -1;
+            merge<false>(st, o);
+            if (un == uy) zy = rec.w;
+        }
+        finalize_row(st, zy, y, ignore, V, eps, out, r, false);
+    }
+}
+
+// dst[c][r] = src[r][c] for a rows x cols bf16 matrix (both 2-byte elements).
+__global__ void __launch_bounds__(256) k_transpose_bf16(const __nv_bfloat16* src, int64_t ld_src,
+                                                        __nv_bfloat16* dst, int64_t ld_dst,
+                                                        int64_t rows, int64_t cols) {
+    __shared__ __nv_bfloat16 tile[64][65];
+    const int64_t tiles_c = (cols + 63) / 64;
+    const int64_t ntiles = ((rows + 63) / 64) * tiles_c;
+    const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 64 x 4
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        const int64_t r0 = (t / tiles_c) * 64, c0 = (t % tiles_c) * 64;
+        for (int i = ty; i < 64; i += 4) {
+            const int64_t r = r0 + i, c = c0 + tx;
+            tile[i][tx] = (r < rows && c < cols) ? src[r * ld_src + c] : __float2bfloat16_rn(0.f);
+        }
+        __syncthreads();
+        for (int i = ty; i < 64; i += 4) {
+            const int64_t c = c0 + i, r = r0 + tx;
+            if (c < cols && r < rows) dst[c * ld_dst + r] = tile[tx][i];
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Tensor map of a row-major bf16 matrix (rows x cols, row stride ld elements)
+// loaded in boxes of 64 columns x box_rows rows with 128-byte swizzle.
+static bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                     int box_rows) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+    cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int EPI>
+static cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmArgs a, int sms,
+                               cudaStream_t s) {
+    static bool attr_set[4] = {false, false, false, false};
+    if (!attr_set[EPI]) {
+        cudaError_t e = cudaFuncSetAttribute(k_gemm<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kGemmSmem);
+        if (e != cudaSuccess) return e;
+        attr_set[EPI] = true;
+    }
+    a.n_mb = (a.M + kBM - 1) / kBM;
+    a.n_nb = (a.Nn + kBN - 1) / kBN;
+    a.nkb = (a.K + kBK - 1) / kBK;
+    if (a.tiles_per_unit < 1) a.tiles_per_unit = 1;
+    a.n_units_n = (a.n_nb + a.tiles_per_unit - 1) / a.tiles_per_unit;
+    a.units = (int64_t)a.n_mb * a.n_units_n;
+    const int grid = (int)(a.units < sms ? a.units : sms);
+    k_gemm<EPI><<<grid, kGemmThreads, kGemmSmem, s>>>(ta, tb, a);
+    return cudaGetLastError();
+}
+
+// Vocabulary tiles per forward unit: a few, so the W tiles in use by all CTAs
+// at once stay in L2 next to H.
+static constexpr int kFwdTilesPerUnit = 4;
+static constexpr int64_t kBwdChunk = 8192;  // vocabulary columns per backward chunk
+
+static int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+static bool linear_shapes_ok(int64_t N, int64_t V, int64_t D, int64_t ld_h, int64_t ld_w) {
+    return N >= 1 && V >= 1 && V <= INT32_MAX && D >= kBK && D % kBK == 0 && ld_h >= D &&
+           ld_w >= D && ld_h % 8 == 0 && ld_w % 8 == 0 && N <= INT32_MAX;
+}
+
+static size_t fwd_ws(int64_t N, int64_t V) {
+    const int64_t n_nb = (V + kBN - 1) / kBN;
+    const int64_t units = (n_nb + kFwdTilesPerUnit - 1) / kFwdTilesPerUnit;
+    return (size_t)units * (size_t)N * sizeof(float4);
+}
+
+struct BwdLayout {
+    size_t off_ht, off_wt, off_g, off_gt, off_acc, total;
+    int64_t ld_ht, ld_wt, vc, ld_gt;
+};
+
+static BwdLayout bwd_layout(int64_t N, int64_t V, int64_t D) {
+    BwdLayout L{};
+    L.ld_ht = round_up(N, 8);
+    L.ld_wt = round_up(V, 8);
+    L.vc = V < kBwdChunk ? round_up(V, kBN) : kBwdChunk;
+    L.ld_gt = round_up(N, 8);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = (size_t)round_up((int64_t)(off + bytes), 256);
+        return o;
+    };
+    L.off_ht = take((size_t)D * L.ld_ht * 2);
+    L.off_wt = take((size_t)D * L.ld_wt * 2);
+    L.off_g = take((size_t)N * L.vc * 2);
+    L.off_gt = take((size_t)L.vc * L.ld_gt * 2);
+    L.off_acc = take((size_t)N * D * 4);
+    L.total = off;
+    return L;
+}
+
+}  // namespace ceb
+
+using namespace ceb;
 
 extern "C" {
 
-size_t linear_ce_workspace_size(int64_t, int64_t, int64_t, int) { return 0; }
-
-ce_status linear_ce_forward(const void*, int64_t, const void*, int64_t, const void*,
-                            ce_index_dtype, int64_t, int64_t, int64_t, float, int64_t,
-                            float*, float*, void*, size_t, void*) {
-    return CE_ENOTSUP;
+size_t linear_ce_workspace_size(int64_t N, int64_t V, int64_t D, int num_sms) {
+    (void)num_sms;
+    (void)D;
+    if (N <= 0 || V <= 0) return 0;
+    return fwd_ws(N, V);
 }
 
-size_t linear_ce_backward_workspace_size(int64_t, int64_t, int64_t, int) { return 0; }
+ce_status linear_ce_forward(const void* H, int64_t ld_h, const void* W, int64_t ld_w,
+                            const void* targets, ce_index_dtype tdt, int64_t N, int64_t V,
+                            int64_t D, float label_smoothing, int64_t ignore_index, float* loss,
+                            float* lse, void* workspace, size_t ws_bytes, void* cuda_stream) {
+    if (!linear_shapes_ok(N, V, D, ld_h, ld_w)) return CE_EINVAL;
+    if (tdt != CE_I32 && tdt != CE_I64) return CE_EINVAL;
+    if (!(label_smoothing >= 0.f && label_smoothing <= 1.f)) return CE_EINVAL;
+    if (!H || !W || !targets || !loss || !lse) return CE_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(H) | reinterpret_cast<uintptr_t>(W)) % 16) return CE_EINVAL;
+    const size_t need = fwd_ws(N, V);
+    if (!workspace || ws_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 16)
+        return CE_EWORKSPACE;
+    unsigned int* err = error_word();
+    if (!err) return CE_ECUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    const int sms = device_sms(0);
 
-ce_status linear_ce_backward(const float*, int64_t, const void*, int64_t, const void*, int64_t,
-                             const void*, ce_index_dtype, const float*, int64_t, int64_t,
-                             int64_t, float, int64_t, void*, ce_dtype, void*, ce_dtype, void*,
-                             size_t, void*) {
-    return CE_ENOTSUP;
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, H, N, D, ld_h, kBM) || !make_map(&tb, W, V, D, ld_w, kBN)) return CE_ECUDA;
+    GemmArgs a{};
+    a.M = (int)N;
+    a.Nn = (int)V;
+    a.K = (int)D;
+    a.tiles_per_unit = kFwdTilesPerUnit;
+    a.err = err;
+    a.y = targets;
+    a.tdt = tdt == CE_I32 ? 0 : 1;
+    a.V = V;
+    a.eps = label_smoothing;
+    a.ignore = ignore_index;
+    a.col_base = 0;
+    a.part = static_cast<float4*>(workspace);
+    if (launch_gemm<kEpiCeFwd>(ta, tb, a, sms, s) != cudaSuccess) return CE_ECUDA;
+    const int64_t n_nb = (V + kBN - 1) / kBN;
+    const int n_units = (int)((n_nb + kFwdTilesPerUnit - 1) / kFwdTilesPerUnit);
+    const int64_t mg = (N + 255) / 256;
+    k_linear_merge<<<(int)(mg < (int64_t)sms * 8 ? mg : (int64_t)sms * 8), 256, 0, s>>>(
+        static_cast<const float4*>(workspace), N, V, kFwdTilesPerUnit * kBN, n_units, targets,
+        a.tdt, label_smoothing, ignore_index, loss, lse, err);
+    return cudaGetLastError() == cudaSuccess ? CE_OK : CE_ECUDA;
+}
+
+size_t linear_ce_backward_workspace_size(int64_t N, int64_t V, int64_t D, int num_sms) {
+    (void)num_sms;
+    if (N <= 0 || V <= 0 || D <= 0) return 0;
+    return bwd_layout(N, V, D).total;
+}
+
+ce_status linear_ce_backward(const float* grad_out, int64_t grad_stride, const void* H,
+                             int64_t ld_h, const void* W, int64_t ld_w, const void* targets,
+                             ce_index_dtype tdt, const float* lse, int64_t N, int64_t V,
+                             int64_t D, float label_smoothing, int64_t ignore_index, void* dH,
+                             ce_dtype dH_dt, void* dW, ce_dtype dW_dt, void* workspace,
+                             size_t ws_bytes, void* cuda_stream) {
+    if (!linear_shapes_ok(N, V, D, ld_h, ld_w)) return CE_EINVAL;
+    if (tdt != CE_I32 && tdt != CE_I64) return CE_EINVAL;
+    if ((dH_dt != CE_BF16 && dH_dt != CE_F32) || (dW_dt != CE_BF16 && dW_dt != CE_F32))
+        return CE_EINVAL;
+    if (!(label_smoothing >= 0.f && label_smoothing <= 1.f)) return CE_EINVAL;
+    if (!grad_out || !H || !W || !targets || !lse || !dH || !dW) return CE_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(H) | reinterpret_cast<uintptr_t>(W) |
+         reinterpret_cast<uintptr_t>(dH) | reinterpret_cast<uintptr_t>(dW)) % 16)
+        return CE_EINVAL;
+    const BwdLayout L = bwd_layout(N, V, D);
+    if (!workspace || ws_bytes < L.total || reinterpret_cast<uintptr_t>(workspace) % 256)
+        return CE_EWORKSPACE;
+    unsigned int* err = error_word();
+    if (!err) return CE_ECUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    const int sms = device_sms(0);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    auto* HT = reinterpret_cast<__nv_bfloat16*>(ws + L.off_ht);
+    auto* WT = reinterpret_cast<__nv_bfloat16*>(ws + L.off_wt);
+    auto* G = reinterpret_cast<__nv_bfloat16*>(ws + L.off_g);
+    auto* GT = reinterpret_cast<__nv_bfloat16*>(ws + L.off_gt);
+    float* dH_acc = dH_dt == CE_F32 ? static_cast<float*>(dH) : reinterpret_cast<float*>(ws + L.off_acc);
+
+    // transposed copies of H and W (K-major operands of the dW and dH passes)
+    {
+        const int64_t t1 = ((N + 63) / 64) * ((D + 63) / 64);
+        const int64_t t2 = ((V + 63) / 64) * ((D + 63) / 64);
+        k_transpose_bf16<<<(int)(t1 < (int64_t)sms * 8 ? t1 : (int64_t)sms * 8), 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(H), ld_h, HT, L.ld_ht, N, D);
+        k_transpose_bf16<<<(int)(t2 < (int64_t)sms * 8 ? t2 : (int64_t)sms * 8), 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(W), ld_w, WT, L.ld_wt, V, D);
+        if (cudaGetLastError() != cudaSuccess) return CE_ECUDA;
+    }
+    CUtensorMap mH, mW, mHT, mWT;
+    if (!make_map(&mH, H, N, D, ld_h, kBM) || !make_map(&mW, W, V, D, ld_w, kBN) ||
+        !make_map(&mHT, HT, D, N, L.ld_ht, kBN) || !make_map(&mWT, WT, D, V, L.ld_wt, kBN))
+        return CE_ECUDA;
+
+    const int64_t nchunks = (V + L.vc - 1) / L.vc;
+    for (int64_t c = 0; c < nchunks; ++c) {
+        const int64_t v0 = c * L.vc;
+        const int64_t vcv = (V - v0) < L.vc ? (V - v0) : L.vc;  // valid columns
+        // GEMM 1: Z_c = H W_c^T, epilogue writes G_c and G_c^T
+        {
+            CUtensorMap mWc;
+            if (!make_map(&mWc, static_cast<const __nv_bfloat16*>(W) + v0 * ld_w, vcv, D, ld_w, kBN))
+                return CE_ECUDA;
+            GemmArgs a{};
+            a.M = (int)N;
+            a.Nn = (int)vcv;
+            a.K = (int)D;
+            a.tiles_per_unit = 1;
+            a.err = err;
+            a.y = targets;
+            a.tdt = tdt == CE_I32 ? 0 : 1;
+            a.V = V;
+            a.eps = label_smoothing;
+            a.ignore = ignore_index;
+            a.col_base = v0;
+            a.g = grad_out;
+            a.g_stride = grad_stride;
+            a.lse = lse;
+            a.G = G;
+            a.ldG = L.vc;
+            a.GT = GT;
+            a.ldGT = L.ld_gt;
+            if (launch_gemm<kEpiCeGrad>(mH, mWc, a, sms, s) != cudaSuccess) return CE_ECUDA;
+        }
+        // GEMM 2: dW[v0:v0+vcv] = G_c^T H  (A = G_c^T, B = H^T, K = N)
+        {
+            CUtensorMap mGT;
+            if (!make_map(&mGT, GT, vcv, N, L.ld_gt, kBM)) return CE_ECUDA;
+            GemmArgs a{};
+            a.M = (int)vcv;
+            a.Nn = (int)D;
+            a.K = (int)N;
+            a.tiles_per_unit = 1;
+            a.err = err;
+            const int esz = dW_dt == CE_F32 ? 4 : 2;
+            a.C = static_cast<uint8_t*>(dW) + (size_t)v0 * D * esz;
+            a.ldc = D;
+            a.c_f32 = dW_dt == CE_F32;
+            if (launch_gemm<kEpiStore>(mGT, mHT, a, sms, s) != cudaSuccess) return CE_ECUDA;
+        }
+        // GEMM 3: dH (+)= G_c W_c  (A = G_c, B = W^T columns [v0, v0+vcv), K = vcv)
+        {
+            CUtensorMap mG;
+            if (!make_map(&mG, G, N, vcv, L.vc, kBM)) return CE_ECUDA;
+            GemmArgs a{};
+            a.M = (int)N;
+            a.Nn = (int)D;
+            a.K = (int)vcv;
+            a.kA0 = 0;
+            a.kB0 = (int)v0;
+            a.tiles_per_unit = 1;
+            a.err = err;
+            a.acc = dH_acc;
+            a.ld_acc = D;
+            a.acc_first = c == 0;
+            a.acc_last = c == nchunks - 1;
+            a.C = dH;
+            a.ldc = D;
+            a.c_f32 = dH_dt == CE_F32;
+            if (launch_gemm<kEpiAccum>(mG, mWT, a, sms, s) != cudaSuccess) return CE_ECUDA;
+        }
+    }
+    return CE_OK;
 }
 
 }  // extern "C"

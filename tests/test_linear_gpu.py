@@ -1,0 +1,138 @@
+"""Fused-linear cross-entropy (Z = H W^T never stored) on the GPU, through
+the C ABI, against the float64 oracle.
+
+Tolerances: the loss within 5e-3 relative of a float64 H W^T (the method's
+statement); we also hold lse to the same bound. dH and dW: normwise relative
+error <= 1e-2 on reduced shapes (the gradient of the logits passes through
+bf16 between the GEMMs), and at full size sampled dH rows against the oracle
+plus two identities that hold at any size: the columns of dW sum to zero
+(every row of the logit gradient sums to zero) and <dH, H> = <dW, W> (both
+equal sum_ij G_ij Z_ij).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+from tests.gpu_util import assert_close, f32, torch
+
+import softmax_cross_entropy_lse_b200 as ce
+from softmax_cross_entropy_lse_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    ce.lib()
+    yield
+    assert ce.get_error() == 0
+
+
+def bf16_dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def run_linear(N, V, D, seed, eps=0.0, ignore_frac=0.0, w_std=0.05, g=None, dtype=torch.float32):
+    hb, hf, wb, wf, y = wl.c5(seed=seed, N=N, V=V, D=D, w_std=w_std)
+    if ignore_frac:
+        rng = np.random.default_rng(seed + 1)
+        y[rng.choice(N, int(ignore_frac * N), replace=False)] = -100
+    H, W, yt = bf16_dev(hb), bf16_dev(wb), torch.from_numpy(y).cuda()
+    loss, lse = ce.linear_ce_forward(H, W, yt, eps)
+    gt = torch.ones(1, device="cuda") if g is None else torch.from_numpy(g).cuda()
+    dH, dW = ce.linear_ce_backward(gt, H, W, yt, lse, eps, dH_dtype=dtype, dW_dtype=dtype)
+    torch.cuda.synchronize()
+    return hf, wf, y, loss, lse, dH, dW
+
+
+def rel_norm(got, ref):
+    return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+@pytest.mark.parametrize("N,V,D", [(128, 256, 64), (512, 8292, 1024), (300, 1000, 256),
+                                   (129, 2049, 192)])
+def test_forward_reduced(orc, N, V, D):
+    hf, wf, y, loss, lse, _, _ = run_linear(N, V, D, seed=N + V + D)
+    ref_loss, ref_lse = orc.linear_ce_forward_rows(hf, wf, y)
+    assert_close(f32(loss), ref_loss, 5e-3, 0.0, "loss")
+    assert_close(f32(lse), ref_lse, 5e-3, 0.0, "lse")
+    # fp32 accumulation of exact bf16 products: far inside the bound
+    assert np.abs(f32(loss) - ref_loss).max() < 1e-3
+
+
+@pytest.mark.parametrize("eps,ignore", [(0.1, 0.1), (0.0, 0.25)])
+def test_forward_smoothing_ignore(orc, eps, ignore):
+    N, V, D = 384, 3000, 512
+    hf, wf, y, loss, lse, _, _ = run_linear(N, V, D, seed=5, eps=eps, ignore_frac=ignore)
+    ref_loss, ref_lse = orc.linear_ce_forward_rows(hf, wf, y, eps=eps)
+    assert_close(f32(loss), ref_loss, 5e-3, 1e-6, "loss")
+    assert_close(f32(lse), ref_lse, 5e-3, 0.0, "lse")
+    assert (f32(loss)[y == -100] == 0).all()
+
+
+@pytest.mark.parametrize("N,V,D,eps", [(256, 1000, 256, 0.0), (200, 777, 128, 0.1),
+                                       (130, 300, 64, 0.0)])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward_reduced(orc, N, V, D, eps, dtype):
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    g = np.random.default_rng(N).standard_normal(N).astype(np.float32) / N
+    hf, wf, y, loss, lse, dH, dW = run_linear(N, V, D, seed=7 + N, eps=eps, ignore_frac=0.1,
+                                              g=g, dtype=dt)
+    rdH, rdW, _ = orc.linear_ce_backward(hf, wf, y, g.astype(np.float64), eps=eps)
+    assert rel_norm(f32(dH).astype(np.float64), rdH) <= 1e-2
+    assert rel_norm(f32(dW).astype(np.float64), rdW) <= 1e-2
+    # ignored rows contribute nothing to dH
+    assert (f32(dH)[y == -100] == 0).all()
+
+
+def test_backward_chunked_vocabulary(orc):
+    """More than one vocabulary chunk (8192 columns each) with a ragged last one."""
+    N, V, D = 160, 8192 + 1000, 128
+    hf, wf, y, loss, lse, dH, dW = run_linear(N, V, D, seed=31, eps=0.1, dtype=torch.float32)
+    rdH, rdW, _ = orc.linear_ce_backward(hf, wf, y, 1.0, eps=0.1)
+    assert rel_norm(f32(dH).astype(np.float64), rdH) <= 1e-2
+    assert rel_norm(f32(dW).astype(np.float64), rdW) <= 1e-2
+
+
+def test_repeat_calls_bitwise_identical():
+    N, V, D = 256, 4096, 512
+    hb, _, wb, _, y = wl.c5(seed=3, N=N, V=V, D=D, w_std=0.05)
+    H, W, yt = bf16_dev(hb), bf16_dev(wb), torch.from_numpy(y).cuda()
+    outs = [ce.linear_ce_forward(H, W, yt) for _ in range(5)]
+    for o in outs[1:]:
+        assert torch.equal(o[0], outs[0][0]) and torch.equal(o[1], outs[0][1])
+    g = torch.ones(1, device="cuda")
+    b0 = ce.linear_ce_backward(g, H, W, yt, outs[0][1], dH_dtype=torch.float32)
+    b1 = ce.linear_ce_backward(g, H, W, yt, outs[0][1], dH_dtype=torch.float32)
+    assert torch.equal(b0[0], b1[0]) and torch.equal(b0[1], b1[1])
+
+
+def test_c5_full_size(orc):
+    """N=8192, V=151,936, D=4096: loss, lse and dH on sampled rows against
+    the oracle; dW through the identities that hold at any size."""
+    N, V, D = 8192, 151936, 4096
+    hb, hf, wb, wf, y = wl.c5()
+    H, W, yt = bf16_dev(hb), bf16_dev(wb), torch.from_numpy(y).cuda()
+    loss, lse = ce.linear_ce_forward(H, W, yt)
+    g = torch.full((1,), 1.0 / N, device="cuda")
+    dH, dW = ce.linear_ce_backward(g, H, W, yt, lse, dH_dtype=torch.float32,
+                                   dW_dtype=torch.float32)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(0).choice(N, 32, replace=False))
+    ref_loss, ref_lse = orc.linear_ce_forward_rows(hf, wf, y, rows=rows)
+    assert_close(f32(loss)[rows], ref_loss, 5e-3, 0.0, "loss")
+    assert_close(f32(lse)[rows], ref_lse, 5e-3, 0.0, "lse")
+    ref_dh = orc.linear_ce_dh_rows(hf, wf, y, 1.0 / N, rows)
+    for k, r in enumerate(rows):
+        assert rel_norm(f32(dH[r]).astype(np.float64), ref_dh[k]) <= 1e-2
+    assert torch.isfinite(loss).all() and torch.isfinite(dW).all()
+    # the columns of dW sum to zero (relative to the size of dW)
+    colsum = dW.double().sum(0)
+    assert (colsum.norm() / dW.double().norm()).item() < 1e-2
+    # <dH, H> = <dW, W>
+    a = (dH.double() * H.double()).sum().item()
+    b = (dW.double() * W.double()).sum().item()
+    assert abs(a - b) <= 1e-2 * max(abs(a), abs(b), 1e-30)
