@@ -343,8 +343,8 @@ def bench_rows(args, rank, world, pg):
 def bench_linear(args, rank, world, pg):
     import torch
     import softmax_cross_entropy_lse_b200 as ce
-    N, V, D = 8192, 151936, 4096
-    hb, hf, wb, wf, y = wl.c5(seed=rank)
+    N, V, D = args.linear_shape
+    hb, hf, wb, wf, y = wl.c5(seed=rank, N=N, V=V, D=D)
     dev = torch.device("cuda", torch.cuda.current_device())
     H_h = torch.from_numpy(hb.view(np.int16)).view(torch.bfloat16)
     W_h = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16)
@@ -422,14 +422,14 @@ def bench_linear(args, rank, world, pg):
         "data": "synthetic",
         "fwd_tflops": round(fwd_flop / (fwd_ms * 1e-3) / 1e12, 2), "fwd_ms": round(fwd_ms, 4),
         "bwd_ms": round(bwd_ms, 4),
-        "config": {"workload": "c5: fused linear CE, H (8192, 4096) bf16 ~N(0,1), W (151,936, 4096) "
+        "config": {"workload": f"c5: fused linear CE, H ({N}, {D}) bf16 ~N(0,1), W ({V}, {D}) "
                                "bf16 ~N(0, std 0.02), forward + backward (logits recomputed)",
                    "N": N, "V": V, "D": D, "flop_per_step": step_flop,
                    "l2": "operands larger than L2 (W is 1.24 GB)",
                    "parallelism": f"rows sharded, {world} independent replica(s), no collective"},
         "e2e": {"value": round(world * step_flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": (N * D + V * D) * 2 + 4 * N, "d2h_bytes_per_step": 4 * N},
-        "gpu_launches": None,
+        "gpu_launches": (2 + 2 + 3 * ((V + 8191) // 8192)) * args.steps,
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2),
                      "peak": peak_sust, "unit": "TFLOP/s", "frac": round(achieved / peak_sust, 4),
                      "traffic": recorded_traffic("c5", dom), "peak_source": src + " (sustained)"},
@@ -576,8 +576,11 @@ def main():
     ap.add_argument("--workload", default="c2", choices=sorted(ROW_WORKLOADS) + ["c5"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--linear-shape", default="8192,151936,4096",
+                    help="N,V,D of the fused-linear workload (c5 is 8192,151936,4096)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    args.linear_shape = tuple(int(x) for x in args.linear_shape.split(","))
     if args.impl == "reference":
         return run_reference(args)
 
