@@ -203,6 +203,8 @@ def bench_rows(args, rank, world, pg):
     spec = ROW_WORKLOADS[args.workload]
     dt, eps = spec["dt"], spec["eps"]
     z, z32, y, kind = make_rows(args.workload, seed=rank)
+    if args.rows and kind == "plain":  # a smaller batch of the same rows (profiling)
+        z, z32, y = z[:args.rows], z32[:args.rows], y[:args.rows]
     dev = torch.device("cuda", torch.cuda.current_device())
     if dt == "bf16":
         z_h = torch.from_numpy(np.ascontiguousarray(z).view(np.int16)).view(torch.bfloat16)
@@ -576,6 +578,8 @@ def main():
     ap.add_argument("--workload", default="c2", choices=sorted(ROW_WORKLOADS) + ["c5"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="use only the first ROWS rows of a row workload (profiling small cases)")
     ap.add_argument("--linear-shape", default="8192,151936,4096",
                     help="N,V,D of the fused-linear workload (c5 is 8192,151936,4096)")
     args = ap.parse_args()

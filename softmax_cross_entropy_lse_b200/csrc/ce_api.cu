@@ -138,14 +138,19 @@ static FwdPlan plan_forward(int64_t N, int64_t V, int esz, bool vec_ok, int sms)
         p.kind = FwdPlan::kPacked;
         const int64_t nvec = V / p.vec;
         p.G = packed_lanes(nvec);
-        p.U = (p.G == 1 && nvec <= 2) ? 2 : 8;
-        const int64_t rows_per_block = 8 * (32 / p.G);
+        p.U = (p.G == 1 && nvec <= 2) ? 2 : (esz == 4 ? 8 : 4);
+        p.R = 1;
+        const int64_t rows_per_block = 8 * (32 / p.G) * p.R;
         const int64_t want = (N + rows_per_block - 1) / rows_per_block;
         const int64_t cap = (int64_t)sms * 16;
         p.grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
         return p;
     }
     p.kind = FwdPlan::kCta;
+    // 2-byte rows fold at twice the elements per byte: their loads go through
+    // bulk-copy rings so that bytes in flight do not depend on registers;
+    // 4-byte rows keep register-staged 16-byte loads, which measured faster
+    p.ring = (vec_ok && esz == 2) ? 1 : 0;
     p.splits = plan_splits(N, V, esz, sms);
     const int64_t nvec = V / p.vec;
     int64_t vps = (nvec + p.splits - 1) / p.splits;
@@ -177,19 +182,33 @@ static BwdPlan plan_backward(int64_t N, int64_t V, int esz_in, bool vec_ok, int 
     BwdPlan p{};
     p.vec = vec_ok ? 16 / esz_in : 1;
     const int64_t nvec = V / p.vec;
+    p.R = 1;
+    p.ring = 0;
+    p.rows = 0;
+    const int kU = p.vec == 1 ? 8 : 32 / p.vec;
     if (nvec <= 256) {
+        p.rows = 1;
         p.G = packed_lanes(nvec);
-        p.U = (p.G == 1 && nvec <= 2) ? 2 : 8;
+        p.U = (p.G == 1 && nvec <= 2) ? 2 : kU;
         *nchunks = 1;
         *vpc = nvec > 0 ? nvec : 1;
     } else {
+        // long rows: one warp per (row, chunk) unit; aligned 2-byte rows stream
+        // through bulk-copy rings, other layouts through register loads
         p.G = 32;
-        p.U = 4;
+        p.U = p.vec == 1 ? 8 : 4;
+        p.ring = (vec_ok && esz_in == 2) ? 1 : 0;
         *vpc = kBwdChunkVecs;
         *nchunks = (nvec + kBwdChunkVecs - 1) / kBwdChunkVecs;
     }
+    if (p.ring) {
+        const int64_t want = (N * *nchunks + 7) / 8;  // 8 warps per CTA
+        const int64_t cap = (int64_t)sms * 2;
+        p.grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
+        return p;
+    }
     const int64_t groups_per_block = 256 / p.G;
-    const int64_t want = (N * *nchunks + groups_per_block - 1) / groups_per_block;
+    const int64_t want = (N * *nchunks + groups_per_block * p.R - 1) / (groups_per_block * p.R);
     const int64_t cap = (int64_t)sms * 16;
     p.grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
     return p;

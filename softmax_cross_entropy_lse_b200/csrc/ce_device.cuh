@@ -149,7 +149,13 @@ __device__ __forceinline__ void store_vec(TO* row, int64_t col, int64_t s_col, c
 }
 
 // ---------------------------------------------------------------------------
-// Online state.
+// Online state: running max m, s = sum_j exp(z_j - m) and t = sum_j (z_j - m)
+// over the k elements seen. Every term is formed from the difference z_j - m
+// first (exact when z_j is near m, by Sterbenz's lemma), then scaled by
+// log2 e for the hardware base-2 exponential: the gap between z_j and m
+// survives at any magnitude (a fused z log2 e - m log2 e would carry the
+// rounding error of m log2 e, which is huge for |m| ~ 1e36). Pairs of
+// elements go through packed f32x2 arithmetic.
 struct OnlineState {
     float m;  // running max (never NaN: fmaxf drops NaN operands)
     float s;  // sum of exp(z - m)
@@ -170,6 +176,12 @@ __device__ __forceinline__ OnlineState empty_state() {
     return st;
 }
 
+__device__ __forceinline__ float lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // True when candidate (bv, bi) should replace (av, ai) as the argmax: a NaN
 // beats any number, a larger value wins, and equal values (or two NaNs) go to
 // the lower index.
@@ -182,12 +194,28 @@ __device__ __forceinline__ bool argmax_better(float bv, int bi, float av, int ai
     return bi < ai;
 }
 
-// Rescale the state to a new max mn >= st.m.
+// Rescale the state to a new max mn >= st.m (st.m = -inf gives factor 0).
 __device__ __forceinline__ void rescale_to(OnlineState& st, float mn) {
     if (st.m != mn) {
-        st.s *= ex2((st.m - mn) * kLog2e);  // st.m = -inf gives 0
+        st.s *= ex2((st.m - mn) * kLog2e);
         if (st.k != 0) st.t += (float)st.k * (st.m - mn);
         st.m = mn;
+    }
+}
+
+// Adds exp(x - ms) and (x - ms) for an even number n of values, two at a
+// time in packed f32x2 arithmetic.
+template <int n>
+__device__ __forceinline__ void accumulate2(const float* x, float ms, float2& sa, float2& ta) {
+    static_assert(n % 2 == 0, "pairs");
+    const float2 l2 = make_float2(kLog2e, kLog2e);
+    const float2 nm = make_float2(-ms, -ms);
+#pragma unroll
+    for (int i = 0; i < n; i += 2) {
+        const float2 d = __fadd2_rn(make_float2(x[i], x[i + 1]), nm);
+        const float2 d2 = __fmul2_rn(d, l2);
+        sa = __fadd2_rn(sa, make_float2(ex2(d2.x), ex2(d2.y)));
+        ta = __fadd2_rn(ta, d);
     }
 }
 
@@ -200,15 +228,19 @@ __device__ __forceinline__ void fold(OnlineState& st, const float* v, int col0, 
     for (int i = 1; i < n; ++i) cm = fmaxf(cm, v[i]);
     rescale_to(st, fmaxf(st.m, cm));
     const float ms = (st.m == -INFINITY) ? 0.f : st.m;
-    float sa = 0.f, ta = 0.f;
+    if constexpr (n % 2 == 0) {
+        float2 sa = make_float2(0.f, 0.f), ta = make_float2(0.f, 0.f);
+        accumulate2<n>(v, ms, sa, ta);
+        st.s += sa.x + sa.y;
+        st.t += ta.x + ta.y;
+    } else {
 #pragma unroll
-    for (int i = 0; i < n; ++i) {
-        const float d = v[i] - ms;
-        sa += ex2(d * kLog2e);
-        ta += d;
+        for (int i = 0; i < n; ++i) {
+            const float d = v[i] - ms;
+            st.s += ex2(d * kLog2e);
+            st.t += d;
+        }
     }
-    st.s += sa;
-    st.t += ta;
     st.k += n;
     if constexpr (ARGMAX) {
 #pragma unroll
@@ -238,24 +270,38 @@ __device__ __forceinline__ void fold_vecs(OnlineState& st, const float (&v)[U][V
     }
     rescale_to(st, fmaxf(st.m, cm));
     const float ms = (st.m == -INFINITY) ? 0.f : st.m;
-    float sa = 0.f, ta = 0.f;
     int n = 0;
+    if constexpr (VEC % 2 == 0) {
+        // one partial pair per vector, then a sum over vectors: short
+        // dependency chains for the adds
+        float2 sa = make_float2(0.f, 0.f), ta = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-        if (MASKED && !ok[u]) continue;
-        float su = 0.f, tu = 0.f;
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-            const float d = v[u][e] - ms;
-            su += ex2(d * kLog2e);
-            tu += d;
+        for (int u = 0; u < U; ++u) {
+            if (MASKED && !ok[u]) continue;
+            float2 su = make_float2(0.f, 0.f), tu = make_float2(0.f, 0.f);
+            accumulate2<VEC>(v[u], ms, su, tu);
+            sa = __fadd2_rn(sa, su);
+            ta = __fadd2_rn(ta, tu);
+            n += VEC;
         }
-        sa += su;
-        ta += tu;
-        n += VEC;
+        st.s += sa.x + sa.y;
+        st.t += ta.x + ta.y;
+    } else {
+        float sa = 0.f, ta = 0.f;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (MASKED && !ok[u]) continue;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+                const float d = v[u][e] - ms;
+                sa += ex2(d * kLog2e);
+                ta += d;
+            }
+            n += VEC;
+        }
+        st.s += sa;
+        st.t += ta;
     }
-    st.s += sa;
-    st.t += ta;
     st.k += n;
 }
 
@@ -335,9 +381,10 @@ __device__ __forceinline__ int64_t load_target(const void* y, int tdt, int64_t o
 }
 
 // ---------------------------------------------------------------------------
-// Finalisation of one row from its complete state.
-//   lse  = m + log s, written as a float pair (hi, lo) with hi + lo = m + L to
-//          about 48 bits (two-sum of m and L = log s);
+// Finalisation of one row from its complete state, with L = log s (hardware
+// base-2 logarithm times ln 2):
+//   lse  = m + L, written as a float pair (hi, lo) with hi + lo = m + L to
+//          about 48 bits (two-sum of m and L);
 //   loss = L - (1-eps)(z_y - m) - eps t/V   (t = sum_j (z_j - m))
 // ignore_index rows: loss 0. Out-of-range targets: loss NaN and error bit 1.
 struct RowOut {
@@ -351,7 +398,7 @@ struct RowOut {
 __device__ __forceinline__ void finalize_row(const OnlineState& st, float zy, int64_t y,
                                              int64_t ignore, int64_t V, float eps,
                                              const RowOut& o, int64_t r, bool write_argmax) {
-    const float L = logf(st.s);
+    const float L = lg2(st.s) * kLn2;  // log sum_j exp(z_j - m)
     const float hi = st.m + L;
     float lo = 0.f;
     if (isfinite(hi)) {

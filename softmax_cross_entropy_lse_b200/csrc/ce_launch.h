@@ -37,6 +37,8 @@ struct FwdPlan {
     enum Kind { kPacked = 0, kCta = 1 } kind;
     int vec;        // 1 (scalar path) or the 16-byte vector width of the dtype
     int G, U;       // packed: lanes per row, vectors per lane per step
+    int R;          // packed: rows per group per step
+    int ring;       // long rows through per-warp bulk-copy rings
     int grid;
     int merge_grid;
     int splits;
@@ -68,6 +70,9 @@ struct BwdArgs {
 struct BwdPlan {
     int vec;
     int G, U;
+    int R;     // units per group per step
+    int ring;  // long rows through per-warp bulk-copy rings
+    int rows;  // short rows, one unit per row (k_bwd_rows)
     int grid;
 };
 

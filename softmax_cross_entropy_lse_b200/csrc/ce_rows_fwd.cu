@@ -17,44 +17,53 @@
 // Ineshin, "A fused linear cross-entropy forward kernel for Apple GPUs", §1.
 #include "ce_device.cuh"
 #include "ce_launch.h"
+#include "ce_sm100.cuh"
 
 namespace ceb {
 
 // ---------------------------------------------------------------------------
-// Packed rows: G lanes per row, U vectors of VEC elements per lane per step.
-template <typename T, int VEC, int G, int U, bool ARGMAX>
-__global__ void __launch_bounds__(256) k_fwd_packed(FwdArgs a) {
+// Packed rows: G lanes per row, U vectors of VEC elements per lane per step,
+// 32/G rows per warp. The lane whose slice holds column y keeps z_y from its
+// registers (no second, dependent load of the row), and the group adds the
+// one nonzero contribution during the reduction.
+template <typename T, int VEC, int G, int U, bool ARGMAX, int MINB>
+__global__ void __launch_bounds__(256, MINB) k_fwd_packed(FwdArgs a) {
     const T* __restrict__ z = reinterpret_cast<const T*>(a.z);
     const int lane = threadIdx.x & 31;
     const int gl = lane & (G - 1);
-    constexpr int kRowsPerWarp = 32 / G;
+    constexpr int kRowsPerStep = 32 / G;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int64_t nvec = a.V / VEC;
     const int tail = (int)(a.V - nvec * VEC);
     const RowOut out{a.loss, a.lse, a.lse_lo, a.argmax, a.err};
 
-    for (int64_t base = warp * kRowsPerWarp; base < a.N; base += nwarps * kRowsPerWarp) {
+    for (int64_t base = warp * kRowsPerStep; base < a.N; base += nwarps * kRowsPerStep) {
         const int64_t r = base + lane / G;
         const bool active = r < a.N;
         OnlineState st = empty_state();
-        int64_t y = 0;
+        int64_t y = a.ignore;
         const T* row = z;
         if (active) {
             row = z + row_offset(a.lz, r, a.N);
             y = load_target(a.y, a.tdt, row_offset(a.ly, r, a.N));
-            for (int64_t vb = 0; vb < nvec; vb += (int64_t)G * U) {
-                float v[U][VEC];
-                bool ok[U];
-                int c0[U];
-                const bool full = vb + (int64_t)G * U <= nvec;
+        }
+        // column of the target logit, or -1 when there is none to capture
+        const int yc = (y >= 0 && y < a.V && y != a.ignore) ? (int)y : -1;
+        float zy = 0.f;
+        for (int64_t vb = 0; vb < nvec; vb += (int64_t)G * U) {
+            float v[U][VEC];
+            bool ok[U];
+            int c0[U];
+            const bool full = vb + (int64_t)G * U <= nvec;
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const int64_t vi = vb + u * G + gl;
-                    ok[u] = full || vi < nvec;
-                    c0[u] = (int)(vi * VEC);
-                    if (ok[u]) load_vec<T, VEC>(row, vi * VEC, a.lz.s_col, v[u]);
-                }
+            for (int u = 0; u < U; ++u) {
+                const int64_t vi = vb + u * G + gl;
+                ok[u] = active && (full || vi < nvec);
+                c0[u] = (int)(vi * VEC);
+                if (ok[u]) load_vec<T, VEC>(row, vi * VEC, a.lz.s_col, v[u]);
+            }
+            if (active) {
                 if (full) {
                     fold_vecs<U, VEC, false>(st, v, ok);
                     if constexpr (ARGMAX) argmax_vecs<U, VEC, false>(st, v, ok, c0);
@@ -62,20 +71,31 @@ __global__ void __launch_bounds__(256) k_fwd_packed(FwdArgs a) {
                     fold_vecs<U, VEC, true>(st, v, ok);
                     if constexpr (ARGMAX) argmax_vecs<U, VEC, true>(st, v, ok, c0);
                 }
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const unsigned dy = (unsigned)(yc - c0[u]);
+                    if (ok[u] && dy < (unsigned)VEC) {
+#pragma unroll
+                        for (int e = 0; e < VEC; ++e)
+                            if ((unsigned)e == dy) zy = v[u][e];
+                    }
+                }
             }
-            // ragged tail: the last V % VEC columns, one per lane
+        }
+        // ragged tail: the last V % VEC columns, one per lane
+        if (active) {
             for (int q = gl; q < tail; q += G) {
                 float x;
-                load_vec<T, 1>(row, nvec * VEC + q, 1, &x);
-                fold<1, ARGMAX>(st, &x, (int)(nvec * VEC + q), 0);
+                const int col = (int)(nvec * VEC + q);
+                load_vec<T, 1>(row, col, 1, &x);
+                fold<1, ARGMAX>(st, &x, col, 0);
+                if (col == yc) zy = x;
             }
         }
         group_reduce<G, ARGMAX>(st);
-        if (active && gl == 0) {
-            float zy = 0.f;
-            if (y != a.ignore && y >= 0 && y < a.V) zy = to_f32(row[y * a.lz.s_col]);
-            finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);
-        }
+#pragma unroll
+        for (int off = G / 2; off >= 1; off >>= 1) zy += __shfl_xor_sync(0xffffffffu, zy, off);
+        if (active && gl == 0) finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);
     }
 }
 
@@ -169,6 +189,211 @@ __global__ void __launch_bounds__(kCtaThreads, kCtaMinBlocks) k_fwd_cta(FwdArgs 
     }
 }
 
+// ---------------------------------------------------------------------------
+// Long rows through per-warp bulk-copy rings. One CTA of kRingWarps warps
+// folds one (row, split) unit, as in k_fwd_cta, but the row reaches shared
+// memory through the tensor-memory-access engine: every warp owns a ring of
+// kRingStages buffers of kRingVecs 16-byte vectors, its lane 0 keeps the ring
+// full with 1-D bulk copies issued kRingStages chunks ahead (across unit
+// boundaries), and the lanes fold each chunk straight from shared memory. The
+// bytes in flight per SM are set by the rings (up to 192 KB), not by the
+// registers of the folding threads. Chunk c of a unit belongs to warp
+// c % kRingWarps; the warps of a unit meet once, in one exchange of states.
+constexpr int kRingWarps = 8;
+constexpr int kRingStages = 6;
+constexpr int kRingVecs = 128;  // 2 KB per stage
+constexpr size_t kRingSmem = (size_t)kRingWarps * kRingStages * kRingVecs * 16;
+
+struct RingUnit {
+    const uint8_t* src;  // first byte of the unit's vectors
+    int64_t v0, nv;      // first vector index in the row, vector count
+    int nch;             // chunks
+};
+
+template <typename T>
+__device__ __forceinline__ RingUnit ring_unit(const FwdArgs& a, int64_t u, int64_t nvec) {
+    RingUnit ru;
+    const int64_t r = a.splits == 1 ? u : u / a.splits;
+    const int64_t sp = a.splits == 1 ? 0 : u - r * a.splits;
+    ru.v0 = sp * a.vec_per_split;
+    const int64_t v1 = min(nvec, ru.v0 + a.vec_per_split);
+    ru.nv = v1 > ru.v0 ? v1 - ru.v0 : 0;
+    ru.nch = (int)((ru.nv + kRingVecs - 1) / kRingVecs);
+    ru.src = reinterpret_cast<const uint8_t*>(reinterpret_cast<const T*>(a.z) +
+                                              row_offset(a.lz, r, a.N)) +
+             ru.v0 * 16;
+    return ru;
+}
+
+// The sequence of (unit, chunk) pairs one warp consumes, in order.
+template <typename T>
+struct RingCursor {
+    int64_t u;
+    int j;
+    RingUnit ru;
+    __device__ __forceinline__ void settle(const FwdArgs& a, int64_t units, int64_t nvec, int w) {
+        while (u < units && j >= ru.nch) {
+            u += gridDim.x;
+            j = w;
+            if (u < units) ru = ring_unit<T>(a, u, nvec);
+        }
+    }
+    __device__ __forceinline__ void start(const FwdArgs& a, int64_t units, int64_t nvec, int w) {
+        u = blockIdx.x;
+        j = w;
+        ru.nch = 0;
+        if (u < units) ru = ring_unit<T>(a, u, nvec);
+        settle(a, units, nvec, w);
+    }
+    __device__ __forceinline__ void next(const FwdArgs& a, int64_t units, int64_t nvec, int w) {
+        j += kRingWarps;
+        settle(a, units, nvec, w);
+    }
+    __device__ __forceinline__ bool valid(int64_t units) const { return u < units; }
+    __device__ __forceinline__ uint32_t bytes() const {
+        const int64_t left = ru.nv - (int64_t)j * kRingVecs;
+        return (uint32_t)((left < kRingVecs ? left : kRingVecs) * 16);
+    }
+    __device__ __forceinline__ const uint8_t* src() const {
+        return ru.src + (int64_t)j * kRingVecs * 16;
+    }
+};
+
+template <typename T, bool ARGMAX>
+__global__ void __launch_bounds__(kRingWarps * 32, 2) k_fwd_ring(FwdArgs a) {
+    using namespace sm100;
+    constexpr int VEC = ElemTraits<T>::kVec;
+    constexpr int kPerLane = kRingVecs / 32;
+    extern __shared__ __align__(128) uint8_t ring_smem[];
+    __shared__ __align__(8) uint64_t full_bar[kRingWarps][kRingStages];
+    __shared__ OnlineState slots[2][kRingWarps];
+    __shared__ int abort_flag;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int64_t nvec = a.V / VEC;
+    const int tail = (int)(a.V - nvec * VEC);
+    const int64_t units = a.N * a.splits;
+    const RowOut out{a.loss, a.lse, a.lse_lo, a.argmax, a.err};
+    uint8_t* ring = ring_smem + (size_t)wid * kRingStages * kRingVecs * 16;
+
+    if (lane == 0)
+        for (int q = 0; q < kRingStages; ++q) mbar_init(smem_u32(&full_bar[wid][q]), 1);
+    if (tid == 0) abort_flag = 0;
+    if (lane == 0) mbar_fence_init();
+    __syncthreads();
+
+    // prologue: the first kRingStages chunks of this warp's sequence
+    RingCursor<T> iss;
+    iss.start(a, units, nvec, wid);
+    int64_t issued = 0;
+    for (int q = 0; q < kRingStages && iss.valid(units); ++q) {
+        if (lane == 0) {
+            const uint32_t bar = smem_u32(&full_bar[wid][q]);
+            mbar_expect_tx(bar, iss.bytes());
+            bulk_load(smem_u32(ring + q * kRingVecs * 16), iss.src(), iss.bytes(), bar);
+        }
+        ++issued;
+        iss.next(a, units, nvec, wid);
+    }
+
+    int64_t consumed = 0, waited = 0;
+    bool dead = false;
+    int parity = 0;
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, parity ^= 1) {
+        const RingUnit ru = ring_unit<T>(a, u, nvec);
+        const int64_t r = a.splits == 1 ? u : u / a.splits;
+        const int sp = a.splits == 1 ? 0 : (int)(u - r * a.splits);
+        const T* row = reinterpret_cast<const T*>(a.z) + row_offset(a.lz, r, a.N);
+        int64_t y = 0;
+        float zy = 0.f;
+        if (a.splits == 1 && tid == 0) {
+            y = load_target(a.y, a.tdt, row_offset(a.ly, r, a.N));
+            if (y != a.ignore && y >= 0 && y < a.V) zy = to_f32(row[y]);
+        }
+        OnlineState st = empty_state();
+        for (int j = wid; j < ru.nch; j += kRingWarps) {
+            const int stage = (int)(consumed % kRingStages);
+            const uint32_t bar = smem_u32(&full_bar[wid][stage]);
+            if (!dead) {
+                if (mbar_wait(bar, (uint32_t)((consumed / kRingStages) & 1), &abort_flag))
+                    ++waited;
+                else
+                    dead = true;
+            }
+            if (!dead) {
+                const int64_t left = ru.nv - (int64_t)j * kRingVecs;
+                const int nvc = (int)(left < kRingVecs ? left : kRingVecs);
+                const uint4* buf = reinterpret_cast<const uint4*>(ring + stage * kRingVecs * 16);
+                float v[kPerLane][VEC];
+                bool ok[kPerLane];
+                int c0[kPerLane];
+#pragma unroll
+                for (int q = 0; q < kPerLane; ++q) {
+                    const int vi = q * 32 + lane;
+                    ok[q] = vi < nvc;
+                    c0[q] = (int)((ru.v0 + (int64_t)j * kRingVecs + vi) * VEC);
+                    if (ok[q]) unpack_words<T>(buf[vi], v[q]);
+                }
+                if (nvc == kRingVecs) {
+                    fold_vecs<kPerLane, VEC, false>(st, v, ok);
+                    if constexpr (ARGMAX) argmax_vecs<kPerLane, VEC, false>(st, v, ok, c0);
+                } else {
+                    fold_vecs<kPerLane, VEC, true>(st, v, ok);
+                    if constexpr (ARGMAX) argmax_vecs<kPerLane, VEC, true>(st, v, ok, c0);
+                }
+            }
+            // the buffer is read: hand it back to the copy engine
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (iss.valid(units) && !dead) {
+                if (lane == 0) {
+                    mbar_expect_tx(bar, iss.bytes());
+                    bulk_load(smem_u32(ring + stage * kRingVecs * 16), iss.src(), iss.bytes(), bar);
+                }
+                ++issued;
+            }
+            iss.next(a, units, nvec, wid);
+            ++consumed;
+        }
+        if (wid == 0 && sp == a.splits - 1) {
+            for (int q = lane; q < tail; q += 32) {
+                float x;
+                load_vec<T, 1>(row, nvec * VEC + q, 1, &x);
+                fold<1, ARGMAX>(st, &x, (int)(nvec * VEC + q), 0);
+            }
+        }
+        group_reduce<32, ARGMAX>(st);
+        if (lane == 0) slots[parity][wid] = st;
+        __syncthreads();
+        if (wid == 0) {
+            st = lane < kRingWarps ? slots[parity][lane] : empty_state();
+            group_reduce<32, ARGMAX>(st);
+            if (lane == 0) {
+                if (a.splits == 1) {
+                    finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);
+                } else {
+                    float4 rec;
+                    rec.x = st.m;
+                    rec.y = st.s;
+                    rec.z = st.t;
+                    const unsigned nanbit = (ARGMAX && st.av != st.av) ? 0x80000000u : 0u;
+                    rec.w = __uint_as_float((unsigned)max(st.ai, 0) | nanbit);
+                    a.part[(int64_t)sp * a.N + r] = rec;
+                }
+            }
+        }
+    }
+    if (dead || abort_flag) {
+        if (lane == 0) atomicOr(a.err, 2u);
+        // let every copy this warp started land before the CTA exits
+        if (lane == 0) {
+            volatile int never = 0;
+            for (int64_t e = waited; e < issued; ++e)
+                mbar_wait(smem_u32(&full_bar[wid][e % kRingStages]), (uint32_t)((e / kRingStages) & 1),
+                          &never);
+        }
+    }
+}
+
 // Merge of split partials, in split order, one thread per row.
 template <typename T, bool ARGMAX>
 __global__ void __launch_bounds__(256) k_fwd_merge(FwdArgs a) {
@@ -209,18 +434,22 @@ __global__ void __launch_bounds__(256) k_fwd_merge(FwdArgs a) {
 
 template <typename T, int VEC, bool ARGMAX>
 static cudaError_t launch_packed(const FwdArgs& a, int G, int U, int grid, cudaStream_t s) {
-#define CEB_PACKED(GG, UU)                                                        \
+    // 32 values per lane per step (8 loads of 4-byte, 4 of 2-byte types);
+    // register budgets for three (4-byte) or two (2-byte) blocks per SM
+    constexpr int kU = sizeof(T) == 4 ? 8 : 4;
+    constexpr int kMinB = sizeof(T) == 4 ? 3 : 2;
+#define CEB_PACKED(GG, UU, MB)                                                    \
     if (G == GG && U == UU) {                                                     \
-        k_fwd_packed<T, VEC, GG, UU, ARGMAX><<<grid, 256, 0, s>>>(a);             \
+        k_fwd_packed<T, VEC, GG, UU, ARGMAX, MB><<<grid, 256, 0, s>>>(a);         \
         return cudaGetLastError();                                                \
     }
-    CEB_PACKED(1, 2)
-    CEB_PACKED(1, 8)
-    CEB_PACKED(2, 8)
-    CEB_PACKED(4, 8)
-    CEB_PACKED(8, 8)
-    CEB_PACKED(16, 8)
-    CEB_PACKED(32, 8)
+    CEB_PACKED(1, 2, kMinB)
+    CEB_PACKED(1, kU, kMinB)
+    CEB_PACKED(2, kU, kMinB)
+    CEB_PACKED(4, kU, kMinB)
+    CEB_PACKED(8, kU, kMinB)
+    CEB_PACKED(16, kU, kMinB)
+    CEB_PACKED(32, kU, kMinB)
 #undef CEB_PACKED
     return cudaErrorInvalidValue;
 }
@@ -232,10 +461,22 @@ static cudaError_t launch_fwd_t(const FwdPlan& p, const FwdArgs& a, cudaStream_t
         return p.vec == 1 ? launch_packed<T, 1, ARGMAX>(a, p.G, p.U, p.grid, s)
                           : launch_packed<T, V8, ARGMAX>(a, p.G, p.U, p.grid, s);
     }
-    if (p.vec == 1)
-        k_fwd_cta<T, 1, 8, ARGMAX><<<p.grid, kCtaThreads, 0, s>>>(a);
-    else
-        k_fwd_cta<T, V8, 4, ARGMAX><<<p.grid, kCtaThreads, 0, s>>>(a);
+    if (!p.ring) {
+        if (p.vec == 1)
+            k_fwd_cta<T, 1, 8, ARGMAX><<<p.grid, kCtaThreads, 0, s>>>(a);
+        else
+            k_fwd_cta<T, V8, 4, ARGMAX><<<p.grid, kCtaThreads, 0, s>>>(a);
+    } else {
+        static bool attr = false;  // per process; the library targets one device per process
+        if (!attr) {
+            cudaError_t e = cudaFuncSetAttribute(k_fwd_ring<T, ARGMAX>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)kRingSmem);
+            if (e != cudaSuccess) return e;
+            attr = true;
+        }
+        k_fwd_ring<T, ARGMAX><<<p.grid, kRingWarps * 32, kRingSmem, s>>>(a);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || a.splits == 1) return e;
     k_fwd_merge<T, ARGMAX><<<p.merge_grid, 256, 0, s>>>(a);
