@@ -275,6 +275,24 @@ def bench_rows(args, rank, world, pg):
     fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
 
+    # the same step through the fused call (one read of each short row)
+    fused_ms = None
+    for i in range(args.warmup):
+        zb, yb, db = bufs[i % nbuf]
+        zvb, yvb = views(zb, yb)
+        ce.ce_forward_backward(zvb, yvb, g, eps, -100, dlogits=views(db, yb)[0], workspace=ws)
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sync_ranks(pg)
+    f0.record(stream)
+    for i in range(args.steps):
+        zb, yb, db = bufs[i % nbuf]
+        zvb, yvb = views(zb, yb)
+        ce.ce_forward_backward(zvb, yvb, g, eps, -100, dlogits=views(db, yb)[0], workspace=ws)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    fused_ms = max_over_ranks(pg, f0.elapsed_time(f1)) / args.steps
+
     # end to end through the public API with host buffers: pinned host inputs
     # copied in, forward + backward, the per-row loss copied out, every step
     z_pin = z_h.pin_memory()
@@ -332,6 +350,13 @@ def bench_rows(args, rank, world, pg):
                      "traffic": recorded_traffic(args.workload, dom),
                      "peak_source": peak_src, "algorithmic_bytes_per_launch": dom_bytes},
     }
+    if fused_ms is not None:
+        fused_bytes = 2 * N * V * esz + 16 * N
+        out["fused"] = {"call": "ce_forward_backward", "ms_per_step": round(fused_ms, 5),
+                        "GB/s": round(fused_bytes / (fused_ms * 1e-3) / 1e9, 2),
+                        "algorithmic_bytes": fused_bytes,
+                        "rows_per_s": round(world * N / (fused_ms * 1e-3), 1),
+                        "speedup_vs_separate": round((ms / args.steps) / fused_ms, 3)}
     if args.workload in PAGE_FWD_BWD_MS:
         page_gbs = step_bytes / (PAGE_FWD_BWD_MS[args.workload] * 1e-3) / 1e9
         out["vs_baseline"] = round(value / page_gbs, 2)

@@ -141,6 +141,29 @@ ce_status ce_backward(const float* grad_out, int64_t grad_stride,
                       void* dlogits, ce_dtype ddt, ce_layout dl,
                       void* cuda_stream);
 
+/* Forward and backward in one call, for when the upstream gradient g is
+ * known before the forward runs (a mean or sum of the per-row losses: g =
+ * 1/count or 1 with grad_stride 0). Writes what ce_forward and ce_backward
+ * write, with the same definitions, readings and errors (argument meanings as
+ * there). Rows short enough for one register step of a warp (up to 1024
+ * elements) are read once: the lanes that fold a row keep it in registers and
+ * write its gradient from them, so the logits cross HBM once instead of
+ * twice. Longer rows run the forward, then the backward.
+ * Sources: Ineshin, "A fused linear cross-entropy forward kernel for Apple
+ * GPUs", section 1 (the backward needs only the row's log-sum-exp, which
+ * the forward has just produced); MLX issue #4686 (the VJP).
+ * dlogits may be the logits themselves (same pointer, dtype and layout); it
+ * must not overlap the per-row outputs or grad_out. The workspace is the
+ * one ce_forward needs for the same shape (only used on the long-row path). */
+ce_status ce_forward_backward(const void* logits, ce_dtype dt, ce_layout lg,
+                              int64_t N, int64_t V,
+                              const void* targets, ce_index_dtype tdt, ce_layout tg,
+                              float label_smoothing, int64_t ignore_index,
+                              const float* grad_out, int64_t grad_stride,
+                              float* loss, float* lse, float* lse_lo, int32_t* argmax,
+                              void* dlogits, ce_dtype ddt, ce_layout dl,
+                              void* workspace, size_t ws_bytes, void* cuda_stream);
+
 /* ------------------------------------------------------------------------ *
  * Fused-linear cross-entropy: logits Z = H W^T are never stored.
  * Source: Ineshin, "A fused linear cross-entropy forward kernel for Apple

@@ -25,7 +25,7 @@ STATUS = {0: "CE_OK", 1: "CE_EINVAL", 2: "CE_EALIAS", 3: "CE_EWORKSPACE", 4: "CE
           5: "CE_ETARGET", 6: "CE_ENOTSUP"}
 EXPORTED = ["ce_workspace_size", "ce_forward", "ce_backward", "linear_ce_workspace_size",
             "linear_ce_forward", "linear_ce_backward_workspace_size", "linear_ce_backward",
-            "ce_get_error", "ce_status_string", "ce_forward_noalloc"]
+            "ce_get_error", "ce_status_string", "ce_forward_noalloc", "ce_forward_backward"]
 NOALLOC_SCRATCH_BYTES = 64 << 10
 
 
@@ -74,6 +74,10 @@ def lib() -> ctypes.CDLL:
         L.ce_forward_noalloc.argtypes = [vp, ctypes.c_int, ce_layout, i64, i64, vp, ctypes.c_int,
                                          ce_layout, f32, i64, vp, vp, vp, vp, vp]
         L.ce_forward_noalloc.restype = ctypes.c_int
+        L.ce_forward_backward.argtypes = [vp, ctypes.c_int, ce_layout, i64, i64, vp, ctypes.c_int,
+                                          ce_layout, f32, i64, vp, i64, vp, vp, vp, vp, vp,
+                                          ctypes.c_int, ce_layout, vp, sz, vp]
+        L.ce_forward_backward.restype = ctypes.c_int
         L.ce_get_error.argtypes = [vp]
         L.ce_get_error.restype = ctypes.c_int
         L.ce_status_string.argtypes = [ctypes.c_int]
@@ -248,6 +252,52 @@ def ce_backward(grad_out, logits, targets, lse, lse_lo=None, label_smoothing: fl
                                _dtype_code(dlogits), dl, _stream(stream))
     _check(st, "ce_backward")
     return dlogits
+
+
+def ce_forward_backward(logits, targets, grad_out, label_smoothing: float = 0.0,
+                        ignore_index: int = -100, *, return_argmax: bool = False, dlogits=None,
+                        out_dtype=None, workspace=None, stream=None):
+    """Forward and VJP in one call (g known up front). Returns (ForwardResult,
+    dlogits); short rows are read from HBM once."""
+    torch = _torch()
+    _require_cuda(logits, targets, grad_out, dlogits)
+    N, lg = row_layout(logits, True)
+    Nt, tg = row_layout(targets, False)
+    if Nt != N:
+        raise ValueError(f"targets hold {Nt} rows, logits {N}")
+    V = logits.shape[-1]
+    if grad_out.dtype != torch.float32:
+        raise TypeError("grad_out must be float32")
+    if grad_out.numel() == 1:
+        g_stride = 0
+    else:
+        if grad_out.numel() != N or grad_out.dim() != 1:
+            raise ValueError("grad_out must hold one value per row (1-D) or a single value")
+        g_stride = grad_out.stride(0)
+    dev = logits.device
+    if dlogits is None:
+        dlogits = torch.empty(logits.shape, dtype=out_dtype or logits.dtype, device=dev)
+    Nd, dl = row_layout(dlogits, True)
+    if Nd != N or dlogits.shape[-1] != V:
+        raise ValueError("dlogits must have the shape of logits")
+    loss = torch.empty(N, dtype=torch.float32, device=dev)
+    lse = torch.empty(N, dtype=torch.float32, device=dev)
+    lse_lo = torch.empty(N, dtype=torch.float32, device=dev)
+    am = torch.empty(N, dtype=torch.int32, device=dev) if return_argmax else None
+    dt = _dtype_code(logits)
+    with torch.cuda.device(dev):
+        need = int(lib().ce_workspace_size(N, V, dt, 0))
+        if workspace is None and need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = lib().ce_forward_backward(_ptr(logits), dt, lg, N, V, _ptr(targets),
+                                       _index_code(targets), tg, float(label_smoothing),
+                                       int(ignore_index), _ptr(grad_out), g_stride, _ptr(loss),
+                                       _ptr(lse), _ptr(lse_lo), _ptr(am), _ptr(dlogits),
+                                       _dtype_code(dlogits), dl, _ptr(workspace), ws_bytes,
+                                       _stream(stream))
+    _check(st, "ce_forward_backward")
+    return ForwardResult(loss, lse, lse_lo, am), dlogits
 
 
 def get_error(stream=None) -> int:

@@ -350,6 +350,103 @@ ce_status ce_backward(const float* grad_out, int64_t grad_stride, const void* lo
     return e == cudaSuccess ? CE_OK : CE_ECUDA;
 }
 
+ce_status ce_forward_backward(const void* logits, ce_dtype dt, ce_layout lg, int64_t N, int64_t V,
+                              const void* targets, ce_index_dtype tdt, ce_layout tg,
+                              float label_smoothing, int64_t ignore_index, const float* grad_out,
+                              int64_t grad_stride, float* loss, float* lse, float* lse_lo,
+                              int32_t* argmax, void* dlogits, ce_dtype ddt, ce_layout dl,
+                              void* workspace, size_t ws_bytes, void* cuda_stream) {
+    if (N < 0 || V < 1 || V > INT32_MAX) return CE_EINVAL;
+    if (dt != CE_F32 && dt != CE_BF16 && dt != CE_F16) return CE_EINVAL;
+    if (ddt != CE_F32 && ddt != dt) return CE_ENOTSUP;
+    if (tdt != CE_I32 && tdt != CE_I64) return CE_EINVAL;
+    if (!(label_smoothing >= 0.f && label_smoothing <= 1.f)) return CE_EINVAL;
+    if (N == 0) return CE_OK;
+    if (!logits || !targets || !loss || !lse || !grad_out || !dlogits) return CE_EINVAL;
+    if (!layout_ok(lg) || !layout_ok(tg) || !layout_ok(dl)) return CE_EINVAL;
+    const int esz = elem_size(dt), dsz = elem_size(ddt);
+    const Layout L = to_layout(lg), T = to_layout(tg), D = to_layout(dl);
+    // the gradient must not overlap the per-row outputs or the upstream gradient
+    const Extent ed = layout_extent(dlogits, D, N, V, dsz);
+    const Extent eg = grad_stride == 0 ? flat_extent(grad_out, 1, 4)
+                                       : layout_extent(grad_out, Layout{N, 0, grad_stride, 0}, N, 1, 4);
+    if (overlap(ed, flat_extent(loss, N, 4)) || overlap(ed, flat_extent(lse, N, 4)) || overlap(ed, eg))
+        return CE_EALIAS;
+    if (lse_lo && overlap(ed, flat_extent(lse_lo, N, 4))) return CE_EALIAS;
+    if (argmax && overlap(ed, flat_extent(argmax, N, 4))) return CE_EALIAS;
+    if (overlap(eg, flat_extent(loss, N, 4)) || overlap(eg, flat_extent(lse, N, 4))) return CE_EALIAS;
+
+    const bool vec_ok = vectorizable(logits, L, N, esz) && vectorizable(dlogits, D, N, dsz);
+    const int vec = vec_ok ? 16 / esz : 1;
+    const int64_t nvec = V / vec;
+    const int kU = vec == 1 ? 8 : 32 / vec;
+    int G = 1;
+    while (G < 32 && nvec > (int64_t)kU * G) G *= 2;
+    if (nvec > (int64_t)kU * G) {
+        // rows longer than one register step of a warp: forward, then the VJP
+        // (which re-reads the logits)
+        ce_status st = ce_forward(logits, dt, lg, N, V, targets, tdt, tg, label_smoothing,
+                                  ignore_index, loss, lse, lse_lo, argmax, workspace, ws_bytes,
+                                  cuda_stream);
+        if (st != CE_OK) return st;
+        return ce_backward(grad_out, grad_stride, logits, dt, lg, N, V, targets, tdt, tg, lse, lse_lo,
+                           label_smoothing, ignore_index, dlogits, ddt, dl, cuda_stream);
+    }
+    // the same checks as the two separate calls
+    {
+        const int tsz = tdt == CE_I32 ? 4 : 8;
+        const Extent ez = layout_extent(logits, L, N, V, esz);
+        const Extent et = layout_extent(targets, Layout{T.inner, T.s_outer, T.s_inner, 0}, N, 1, tsz);
+        Extent outs[4];
+        int nout = 0;
+        outs[nout++] = flat_extent(loss, N, 4);
+        outs[nout++] = flat_extent(lse, N, 4);
+        if (lse_lo) outs[nout++] = flat_extent(lse_lo, N, 4);
+        if (argmax) outs[nout++] = flat_extent(argmax, N, 4);
+        for (int i = 0; i < nout; ++i) {
+            if (overlap(outs[i], ez) || overlap(outs[i], et)) return CE_EALIAS;
+            for (int j = 0; j < i; ++j)
+                if (overlap(outs[i], outs[j])) return CE_EALIAS;
+        }
+        const bool in_place = dlogits == logits && ddt == dt && L.inner == D.inner &&
+                              L.s_outer == D.s_outer && L.s_inner == D.s_inner && L.s_col == D.s_col;
+        if (!in_place && overlap(ed, ez)) return CE_EALIAS;
+        if (overlap(ed, et)) return CE_EALIAS;
+    }
+    const int sms = device_sms(0);
+    FusedPlan p{};
+    p.vec = vec;
+    p.G = G;
+    p.U = (G == 1 && nvec <= 2) ? 2 : kU;
+    const int64_t rows_per_block = 8 * (32 / G);
+    const int64_t want = (N + rows_per_block - 1) / rows_per_block;
+    const int64_t cap = (int64_t)sms * 16;
+    p.grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
+    FusedArgs a{};
+    a.f.z = logits;
+    a.f.N = N;
+    a.f.V = V;
+    a.f.y = targets;
+    a.f.tdt = tdt == CE_I32 ? 0 : 1;
+    a.f.eps = label_smoothing;
+    a.f.ignore = ignore_index;
+    a.f.loss = loss;
+    a.f.lse = lse;
+    a.f.lse_lo = lse_lo;
+    a.f.argmax = argmax;
+    a.f.err = error_word();
+    if (!a.f.err) return CE_ECUDA;
+    a.f.splits = 1;
+    a.f.lz = L;
+    a.f.ly = T;
+    a.g = grad_out;
+    a.g_stride = grad_stride;
+    a.dz = dlogits;
+    a.ld = D;
+    cudaError_t e = launch_fused(p, a, (int)dt, (int)ddt, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? CE_OK : CE_ECUDA;
+}
+
 ce_status ce_get_error(void* cuda_stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess) return CE_ECUDA;
     unsigned int w = 0;

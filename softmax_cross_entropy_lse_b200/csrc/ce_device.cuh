@@ -395,17 +395,25 @@ struct RowOut {
     unsigned int* err;
 };
 
+// L = log sum_j exp(z_j - m) and the float pair (hi, lo) of m + L. Explicit
+// round-to-nearest operations (never contracted into fmas), so every kernel
+// that derives the pair from the same state gets the same bits.
+__device__ __forceinline__ void lse_pair(const OnlineState& st, float& L, float& hi, float& lo) {
+    L = __fmul_rn(lg2(st.s), kLn2);
+    hi = __fadd_rn(st.m, L);
+    lo = 0.f;
+    if (isfinite(hi)) {
+        const float bv = __fsub_rn(hi, st.m);
+        const float av = __fsub_rn(hi, bv);
+        lo = __fadd_rn(__fsub_rn(st.m, av), __fsub_rn(L, bv));
+    }
+}
+
 __device__ __forceinline__ void finalize_row(const OnlineState& st, float zy, int64_t y,
                                              int64_t ignore, int64_t V, float eps,
                                              const RowOut& o, int64_t r, bool write_argmax) {
-    const float L = lg2(st.s) * kLn2;  // log sum_j exp(z_j - m)
-    const float hi = st.m + L;
-    float lo = 0.f;
-    if (isfinite(hi)) {
-        const float bv = hi - st.m;
-        const float av = hi - bv;
-        lo = (st.m - av) + (L - bv);
-    }
+    float L, hi, lo;
+    lse_pair(st, L, hi, lo);
     o.lse[r] = hi;
     if (o.lse_lo) o.lse_lo[r] = lo;
     float loss;

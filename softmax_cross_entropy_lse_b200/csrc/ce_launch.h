@@ -79,4 +79,22 @@ struct BwdPlan {
 cudaError_t launch_backward(const BwdPlan& p, const BwdArgs& a, int dt_in, int dt_out,
                             cudaStream_t s);
 
+// ---- fused forward + backward (short rows) ---------------------------------
+struct FusedArgs {
+    FwdArgs f;
+    const float* g;
+    int64_t g_stride;
+    void* dz;
+    Layout ld;
+};
+
+struct FusedPlan {
+    int vec;
+    int G, U;
+    int grid;
+};
+
+cudaError_t launch_fused(const FusedPlan& p, const FusedArgs& a, int dt_in, int dt_out,
+                         cudaStream_t s);
+
 }  // namespace ceb

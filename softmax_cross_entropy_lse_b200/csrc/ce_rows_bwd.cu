@@ -486,7 +486,10 @@ static cudaError_t launch_bwd_rows(const BwdPlan& p, const BwdArgs& a, cudaStrea
         k_bwd_rows<TI, TO, VEC, GG, UU, kMinB><<<p.grid, 256, 0, s>>>(a);  \
         return cudaGetLastError();                                         \
     }
-    CEB_BWDR(1, 2)
+    if (p.G == 1 && p.U == 2) {  // tiny rows: latency-bound, so as many warps as fit
+        k_bwd_rows<TI, TO, VEC, 1, 2, sizeof(TI) == 4 ? 6 : 4><<<p.grid, 256, 0, s>>>(a);
+        return cudaGetLastError();
+    }
     CEB_BWDR(1, kU)
     CEB_BWDR(2, kU)
     CEB_BWDR(4, kU)

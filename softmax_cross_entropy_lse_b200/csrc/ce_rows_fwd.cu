@@ -443,7 +443,7 @@ static cudaError_t launch_packed(const FwdArgs& a, int G, int U, int grid, cudaS
         k_fwd_packed<T, VEC, GG, UU, ARGMAX, MB><<<grid, 256, 0, s>>>(a);         \
         return cudaGetLastError();                                                \
     }
-    CEB_PACKED(1, 2, kMinB)
+    CEB_PACKED(1, 2, 5)  // tiny rows: latency-bound, so as many warps as fit
     CEB_PACKED(1, kU, kMinB)
     CEB_PACKED(2, kU, kMinB)
     CEB_PACKED(4, kU, kMinB)
