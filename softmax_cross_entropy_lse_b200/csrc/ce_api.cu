@@ -159,7 +159,7 @@ static FwdPlan plan_forward(int64_t N, int64_t V, int esz, bool vec_ok, int sms)
     if (p.splits < 1) p.splits = 1;
     p.vec_per_split = vps;
     const int64_t units = N * p.splits;
-    const int64_t cap = (int64_t)sms * 2;
+    const int64_t cap = (int64_t)sms * (p.ring ? 3 : 2);
     p.grid = (int)(units < cap ? units : cap);
     const int64_t mg = (N + 255) / 256;
     p.merge_grid = (int)(mg < (int64_t)sms * 8 ? mg : (int64_t)sms * 8);

@@ -305,6 +305,76 @@ __device__ __forceinline__ void fold_vecs(OnlineState& st, const float (&v)[U][V
     st.k += n;
 }
 
+// ---- 16-bit rows folded from their raw words -----------------------------------
+// The max is taken with packed 16-bit max instructions on the stored words
+// (exact: every 16-bit value is a float), and the words are widened to float
+// pairs only when their exponentials are formed, so a lane holds its 16-bit
+// data in half the registers. Packed 16-bit max returns the number when one
+// operand is NaN, like fmaxf; the NaN still reaches the sum.
+template <typename T> struct Raw16;
+template <> struct Raw16<__nv_bfloat16> {
+    static constexpr uint32_t kNegInf2 = 0xff80ff80u;
+    static __device__ __forceinline__ uint32_t max2(uint32_t a, uint32_t b) {
+        __nv_bfloat162 r = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                                   *reinterpret_cast<__nv_bfloat162*>(&b));
+        return *reinterpret_cast<uint32_t*>(&r);
+    }
+    static __device__ __forceinline__ float2 widen(uint32_t w) {
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+};
+template <> struct Raw16<__half> {
+    static constexpr uint32_t kNegInf2 = 0xfc00fc00u;
+    static __device__ __forceinline__ uint32_t max2(uint32_t a, uint32_t b) {
+        __half2 r = __hmax2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+        return *reinterpret_cast<uint32_t*>(&r);
+    }
+    static __device__ __forceinline__ float2 widen(uint32_t w) {
+        return __half22float2(*reinterpret_cast<__half2*>(&w));
+    }
+};
+
+// Folds U 16-byte words of 8 16-bit values (valid where ok[u], or all when
+// not MASKED). WITH_T = false skips sum (z - m), which only label smoothing
+// reads.
+template <typename T, int U, bool MASKED, bool WITH_T>
+__device__ __forceinline__ void fold_raw16(OnlineState& st, const uint4 (&w)[U],
+                                           const bool (&ok)[U]) {
+    using R = Raw16<T>;
+    uint32_t mx = R::kNegInf2;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        if (MASKED && !ok[u]) continue;
+        mx = R::max2(mx, R::max2(R::max2(w[u].x, w[u].y), R::max2(w[u].z, w[u].w)));
+    }
+    const float2 m2 = R::widen(mx);
+    rescale_to(st, fmaxf(st.m, fmaxf(m2.x, m2.y)));
+    const float ms = (st.m == -INFINITY) ? 0.f : st.m;
+    const float2 l2 = make_float2(kLog2e, kLog2e);
+    const float2 nm = make_float2(-ms, -ms);
+    float2 sa = make_float2(0.f, 0.f), ta = make_float2(0.f, 0.f);
+    int n = 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        if (MASKED && !ok[u]) continue;
+        const uint32_t ws[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+        float2 su = make_float2(0.f, 0.f), tu = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 d = __fadd2_rn(R::widen(ws[k]), nm);
+            const float2 d2 = __fmul2_rn(d, l2);
+            su = __fadd2_rn(su, make_float2(ex2(d2.x), ex2(d2.y)));
+            if constexpr (WITH_T) tu = __fadd2_rn(tu, d);
+        }
+        sa = __fadd2_rn(sa, su);
+        if constexpr (WITH_T) ta = __fadd2_rn(ta, tu);
+        n += 8;
+    }
+    st.s += sa.x + sa.y;
+    if constexpr (WITH_T) st.t += ta.x + ta.y;
+    st.k += n;
+}
+
 // Argmax over U vectors whose first columns are col0[u], in increasing
 // column order per thread (a strict comparison keeps the first of equals).
 template <int U, int VEC, bool MASKED>

@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(kCtaThreads, kCtaMinBlocks) k_fwd_cta(FwdArgs 
 // registers of the folding threads. Chunk c of a unit belongs to warp
 // c % kRingWarps; the warps of a unit meet once, in one exchange of states.
 constexpr int kRingWarps = 8;
-constexpr int kRingStages = 6;
+constexpr int kRingStages = 4;
 constexpr int kRingVecs = 128;  // 2 KB per stage
 constexpr size_t kRingSmem = (size_t)kRingWarps * kRingStages * kRingVecs * 16;
 
@@ -259,8 +259,8 @@ struct RingCursor {
     }
 };
 
-template <typename T, bool ARGMAX>
-__global__ void __launch_bounds__(kRingWarps * 32, 2) k_fwd_ring(FwdArgs a) {
+template <typename T, bool ARGMAX, bool WITH_T>
+__global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
     using namespace sm100;
     constexpr int VEC = ElemTraits<T>::kVec;
     constexpr int kPerLane = kRingVecs / 32;
@@ -323,22 +323,38 @@ __global__ void __launch_bounds__(kRingWarps * 32, 2) k_fwd_ring(FwdArgs a) {
                 const int64_t left = ru.nv - (int64_t)j * kRingVecs;
                 const int nvc = (int)(left < kRingVecs ? left : kRingVecs);
                 const uint4* buf = reinterpret_cast<const uint4*>(ring + stage * kRingVecs * 16);
-                float v[kPerLane][VEC];
-                bool ok[kPerLane];
-                int c0[kPerLane];
+                if constexpr (sizeof(T) == 2 && !ARGMAX) {
+                    // raw 16-bit words: packed max, widened pairwise for the sum
+                    uint4 w[kPerLane];
+                    bool ok[kPerLane];
 #pragma unroll
-                for (int q = 0; q < kPerLane; ++q) {
-                    const int vi = q * 32 + lane;
-                    ok[q] = vi < nvc;
-                    c0[q] = (int)((ru.v0 + (int64_t)j * kRingVecs + vi) * VEC);
-                    if (ok[q]) unpack_words<T>(buf[vi], v[q]);
-                }
-                if (nvc == kRingVecs) {
-                    fold_vecs<kPerLane, VEC, false>(st, v, ok);
-                    if constexpr (ARGMAX) argmax_vecs<kPerLane, VEC, false>(st, v, ok, c0);
+                    for (int q = 0; q < kPerLane; ++q) {
+                        const int vi = q * 32 + lane;
+                        ok[q] = vi < nvc;
+                        if (ok[q]) w[q] = buf[vi];
+                    }
+                    if (nvc == kRingVecs)
+                        fold_raw16<T, kPerLane, false, WITH_T>(st, w, ok);
+                    else
+                        fold_raw16<T, kPerLane, true, WITH_T>(st, w, ok);
                 } else {
-                    fold_vecs<kPerLane, VEC, true>(st, v, ok);
-                    if constexpr (ARGMAX) argmax_vecs<kPerLane, VEC, true>(st, v, ok, c0);
+                    float v[kPerLane][VEC];
+                    bool ok[kPerLane];
+                    int c0[kPerLane];
+#pragma unroll
+                    for (int q = 0; q < kPerLane; ++q) {
+                        const int vi = q * 32 + lane;
+                        ok[q] = vi < nvc;
+                        c0[q] = (int)((ru.v0 + (int64_t)j * kRingVecs + vi) * VEC);
+                        if (ok[q]) unpack_words<T>(buf[vi], v[q]);
+                    }
+                    if (nvc == kRingVecs) {
+                        fold_vecs<kPerLane, VEC, false>(st, v, ok);
+                        if constexpr (ARGMAX) argmax_vecs<kPerLane, VEC, false>(st, v, ok, c0);
+                    } else {
+                        fold_vecs<kPerLane, VEC, true>(st, v, ok);
+                        if constexpr (ARGMAX) argmax_vecs<kPerLane, VEC, true>(st, v, ok, c0);
+                    }
                 }
             }
             // the buffer is read: hand it back to the copy engine
@@ -454,6 +470,20 @@ static cudaError_t launch_packed(const FwdArgs& a, int G, int U, int grid, cudaS
     return cudaErrorInvalidValue;
 }
 
+template <typename T, bool ARGMAX, bool WITH_T>
+static cudaError_t launch_ring(const FwdPlan& p, const FwdArgs& a, cudaStream_t s) {
+    static bool attr = false;  // per process; the library targets one device per process
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(k_fwd_ring<T, ARGMAX, WITH_T>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kRingSmem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    k_fwd_ring<T, ARGMAX, WITH_T><<<p.grid, kRingWarps * 32, kRingSmem, s>>>(a);
+    return cudaGetLastError();
+}
+
 template <typename T, bool ARGMAX>
 static cudaError_t launch_fwd_t(const FwdPlan& p, const FwdArgs& a, cudaStream_t s) {
     constexpr int V8 = ElemTraits<T>::kVec;
@@ -466,16 +496,12 @@ static cudaError_t launch_fwd_t(const FwdPlan& p, const FwdArgs& a, cudaStream_t
             k_fwd_cta<T, 1, 8, ARGMAX><<<p.grid, kCtaThreads, 0, s>>>(a);
         else
             k_fwd_cta<T, V8, 4, ARGMAX><<<p.grid, kCtaThreads, 0, s>>>(a);
+    } else if (a.eps != 0.f) {
+        cudaError_t e = launch_ring<T, ARGMAX, true>(p, a, s);
+        if (e != cudaSuccess) return e;
     } else {
-        static bool attr = false;  // per process; the library targets one device per process
-        if (!attr) {
-            cudaError_t e = cudaFuncSetAttribute(k_fwd_ring<T, ARGMAX>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)kRingSmem);
-            if (e != cudaSuccess) return e;
-            attr = true;
-        }
-        k_fwd_ring<T, ARGMAX><<<p.grid, kRingWarps * 32, kRingSmem, s>>>(a);
+        cudaError_t e = launch_ring<T, ARGMAX, false>(p, a, s);
+        if (e != cudaSuccess) return e;
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || a.splits == 1) return e;
