@@ -31,6 +31,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from softmax_cross_entropy_lse_b200 import sharding  # noqa: E402
 from softmax_cross_entropy_lse_b200 import workloads as wl  # noqa: E402
 
 METRIC = "CE fwd and fwd+bwd GB/s and rows/s vs HBM roofline; fused-linear TFLOP/s"
@@ -143,39 +144,12 @@ class ClockSampler:
                 "samples": len(rows), "power_w_max": float(max(r[2] for r in rows))}
 
 
-# -- distributed plumbing ---------------------------------------------------------------
+# -- distributed plumbing (softmax_cross_entropy_lse_b200.sharding) --------------------------------
 def dist_setup(n_gpus: int):
-    import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1 and world != n_gpus:
         raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-        pg = dist
-    else:
-        torch.cuda.set_device(0)
-    return rank, world, local, pg
-
-
-def sync_ranks(pg):
-    if pg is not None:
-        pg.barrier()
-
-
-def max_over_ranks(pg, x: float) -> float:
-    if pg is None:
-        return x
-    import torch
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    return float(t.item())
+    return sharding.init_from_env("nccl", timeout_s=120)
 
 
 # -- row workloads ------------------------------------------------------------------------
@@ -197,12 +171,13 @@ def make_rows(workload: str, seed: int):
     return z, z32, y, "plain"
 
 
-def bench_rows(args, rank, world, pg):
+def bench_rows(args, rk):
     import torch
     import softmax_cross_entropy_lse_b200 as ce
+    world = rk.world
     spec = ROW_WORKLOADS[args.workload]
     dt, eps = spec["dt"], spec["eps"]
-    z, z32, y, kind = make_rows(args.workload, seed=rank)
+    z, z32, y, kind = make_rows(args.workload, seed=rk.rank)
     if args.rows and kind == "plain":  # a smaller batch of the same rows (profiling)
         z, z32, y = z[:args.rows], z32[:args.rows], y[:args.rows]
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -221,8 +196,9 @@ def bench_rows(args, rank, world, pg):
     V = zv.shape[-1]
     esz = zv.element_size()
     yflat = (y[:, 1:] if kind == "view" else y).reshape(-1)
-    n_valid = int((yflat != -100).sum())
-    g = torch.full((1,), 1.0 / max(n_valid, 1), dtype=torch.float32, device=dev)  # mean
+    # the mean over the global batch: every rank scales by 1 / (rows counted on
+    # all ranks), one all-reduce of an integer when the batch is formed
+    g = torch.full((1,), sharding.mean_grad_scale(rk, yflat), dtype=torch.float32, device=dev)
     dz = torch.empty(z_d.shape, dtype=z_d.dtype, device=dev)
     dzv = views(dz, y_d)[0]
     ws_bytes = ce.ce_workspace_size(N, V, zv.dtype)
@@ -263,15 +239,15 @@ def bench_rows(args, rank, world, pg):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index) as clk:
-        sync_ranks(pg)
+        sharding.barrier(rk)
         torch.cuda.synchronize()
         t0.record(stream)
         for i in range(args.steps):
             step(i, evs[i])
         t1.record(stream)
         torch.cuda.synchronize()
-        sync_ranks(pg)
-    ms = max_over_ranks(pg, t0.elapsed_time(t1))
+        sharding.barrier(rk)
+    ms = sharding.max_over_ranks(rk, t0.elapsed_time(t1))
     fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
 
@@ -283,7 +259,7 @@ def bench_rows(args, rank, world, pg):
         ce.ce_forward_backward(zvb, yvb, g, eps, -100, dlogits=views(db, yb)[0], workspace=ws)
     torch.cuda.synchronize()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sync_ranks(pg)
+    sharding.barrier(rk)
     f0.record(stream)
     for i in range(args.steps):
         zb, yb, db = bufs[i % nbuf]
@@ -291,7 +267,7 @@ def bench_rows(args, rank, world, pg):
         ce.ce_forward_backward(zvb, yvb, g, eps, -100, dlogits=views(db, yb)[0], workspace=ws)
     f1.record(stream)
     torch.cuda.synchronize()
-    fused_ms = max_over_ranks(pg, f0.elapsed_time(f1)) / args.steps
+    fused_ms = sharding.max_over_ranks(rk, f0.elapsed_time(f1)) / args.steps
 
     # end to end through the public API with host buffers: pinned host inputs
     # copied in, forward + backward, the per-row loss copied out, every step
@@ -311,14 +287,14 @@ def bench_rows(args, rank, world, pg):
     for _ in range(2):
         e2e_step()
     torch.cuda.synchronize()
-    sync_ranks(pg)
+    sharding.barrier(rk)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for _ in range(e2e_steps):
         e2e_step()
     b.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(pg, a.elapsed_time(b)) / e2e_steps
+    e2e_ms = sharding.max_over_ranks(rk, a.elapsed_time(b)) / e2e_steps
     h2d = z_h.numel() * z_h.element_size() + y_h.numel() * y_h.element_size()
     d2h = 4 * N
 
@@ -341,7 +317,7 @@ def bench_rows(args, rank, world, pg):
                    "bytes_per_step": step_bytes,
                    "l2": ("inputs larger than L2" if nbuf == 1 else
                           f"{nbuf} rotating input buffers (total larger than L2)"),
-                   "parallelism": f"rows sharded, {world} independent replica(s), no collective"},
+                   "parallelism": f"rows sharded over {world} rank(s), no data-path collective"},
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
@@ -367,17 +343,18 @@ def bench_rows(args, rank, world, pg):
 
 
 # -- fused-linear workload -------------------------------------------------------------------
-def bench_linear(args, rank, world, pg):
+def bench_linear(args, rk):
     import torch
     import softmax_cross_entropy_lse_b200 as ce
+    world = rk.world
     N, V, D = args.linear_shape
-    hb, hf, wb, wf, y = wl.c5(seed=rank, N=N, V=V, D=D)
+    hb, hf, wb, wf, y = wl.c5(seed=rk.rank, N=N, V=V, D=D)
     dev = torch.device("cuda", torch.cuda.current_device())
     H_h = torch.from_numpy(hb.view(np.int16)).view(torch.bfloat16)
     W_h = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16)
     y_h = torch.from_numpy(y)
     H, W, yd = H_h.to(dev), W_h.to(dev), y_h.to(dev)
-    g = torch.full((1,), 1.0 / N, dtype=torch.float32, device=dev)
+    g = torch.full((1,), sharding.mean_grad_scale(rk, y), dtype=torch.float32, device=dev)
     L = ce.lib()
     ws_f = torch.empty(max(L.linear_ce_workspace_size(N, V, D, 0), 16), dtype=torch.uint8,
                        device=dev)
@@ -403,15 +380,15 @@ def bench_linear(args, rank, world, pg):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index) as clk:
-        sync_ranks(pg)
+        sharding.barrier(rk)
         torch.cuda.synchronize()
         t0.record(stream)
         for i in range(args.steps):
             step(evs[i])
         t1.record(stream)
         torch.cuda.synchronize()
-        sync_ranks(pg)
-    ms = max_over_ranks(pg, t0.elapsed_time(t1))
+        sharding.barrier(rk)
+    ms = sharding.max_over_ranks(rk, t0.elapsed_time(t1))
     fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
     _, peak_burst, peak_sust, src = load_peaks()
@@ -431,14 +408,14 @@ def bench_linear(args, rank, world, pg):
 
     e2e_step()
     torch.cuda.synchronize()
-    sync_ranks(pg)
+    sharding.barrier(rk)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for _ in range(2):
         e2e_step()
     b.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(pg, a.elapsed_time(b)) / 2
+    e2e_ms = sharding.max_over_ranks(rk, a.elapsed_time(b)) / 2
     dom, dom_ms, dom_flop = ("backward", bwd_ms, bwd_flop) if bwd_ms >= fwd_ms else \
         ("forward", fwd_ms, fwd_flop)
     achieved = dom_flop / (dom_ms * 1e-3) / 1e12
@@ -453,7 +430,7 @@ def bench_linear(args, rank, world, pg):
                                "bf16 ~N(0, std 0.02), forward + backward (logits recomputed)",
                    "N": N, "V": V, "D": D, "flop_per_step": step_flop,
                    "l2": "operands larger than L2 (W is 1.24 GB)",
-                   "parallelism": f"rows sharded, {world} independent replica(s), no collective"},
+                   "parallelism": f"rows sharded over {world} rank(s), no data-path collective"},
         "e2e": {"value": round(world * step_flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": (N * D + V * D) * 2 + 4 * N, "d2h_bytes_per_step": 4 * N},
         "gpu_launches": (2 + 2 + 3 * ((V + 8191) // 8192)) * args.steps,
@@ -616,19 +593,19 @@ def main():
     import torch
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
-    rank, world, local, pg = dist_setup(args.gpus)
+    rk = dist_setup(args.gpus)
     if args.workload == "c5":
-        out, host = bench_linear(args, rank, world, pg)
+        out, host = bench_linear(args, rk)
     else:
-        out, host = bench_rows(args, rank, world, pg)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out, host = bench_rows(args, rk)
+    if rk.rank == 0 and rk.world == 1 and not args.no_cpu_baseline:
         v, unit, cores, sample = oracle_baseline(args.workload, 12.0, host)
         out["cpu_baseline"] = {"value": round(v, 4), "unit": unit, "cores": cores,
                                "kind": "oracle", "sample": sample}
-    if pg is not None:
-        pg.barrier()
-        pg.destroy_process_group()
-    if rank == 0:
+    if rk.group is not None:
+        rk.group.barrier()
+        rk.group.destroy_process_group()
+    if rk.rank == 0:
         print(json.dumps(out), flush=True)
     return 0
 
