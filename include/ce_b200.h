@@ -145,10 +145,14 @@ ce_status ce_backward(const float* grad_out, int64_t grad_stride,
  * known before the forward runs (a mean or sum of the per-row losses: g =
  * 1/count or 1 with grad_stride 0). Writes what ce_forward and ce_backward
  * write, with the same definitions, readings and errors (argument meanings as
- * there). Rows short enough for one register step of a warp (up to 1024
- * elements) are read once: the lanes that fold a row keep it in registers and
- * write its gradient from them, so the logits cross HBM once instead of
- * twice. Longer rows run the forward, then the backward.
+ * there). The logits cross HBM once instead of twice wherever a row fits on
+ * chip: rows of up to 1024 elements stay in the registers of the lanes that
+ * fold them; longer rows with 16-byte aligned, unit-stride rows (logits and
+ * dlogits) and up to 8 x 112 KB per row are copied into shared memory, split
+ * over a cluster of 1, 2, 4 or 8 CTAs whose partial states meet once in
+ * distributed shared memory, and differentiated from there. Those rows need
+ * at least (number of SMs / cluster size) rows per call; otherwise, and for
+ * longer or unaligned rows, the call runs the forward, then the backward.
  * Sources: Ineshin, "A fused linear cross-entropy forward kernel for Apple
  * GPUs", section 1 (the backward needs only the row's log-sum-exp, which
  * the forward has just produced); MLX issue #4686 (the VJP).

@@ -382,7 +382,27 @@ ce_status ce_forward_backward(const void* logits, ce_dtype dt, ce_layout lg, int
     const int kU = vec == 1 ? 8 : 32 / vec;
     int G = 1;
     while (G < 32 && nvec > (int64_t)kU * G) G *= 2;
-    if (nvec > (int64_t)kU * G) {
+    const int sms = device_sms(0);
+    // rows beyond one warp's registers: held in shared memory by a cluster of
+    // the fewest CTAs whose slices fit (needs 16-byte rows, and enough rows
+    // to give every SM a CTA); else a forward, then the VJP
+    SmemRowPlan sp{};
+    if (nvec > (int64_t)kU * G && vec_ok) {
+        for (int cl = 1; cl <= 8; cl *= 2) {
+            const int64_t per = (nvec + cl - 1) / cl;
+            const int64_t nch = (per + 127) / 128;
+            if (nch <= kSmemRowMaxChunks) {
+                if (N * cl >= sms) {
+                    sp.cl = cl;
+                    sp.nch = (int)nch;
+                    sp.vec_per_cta = per;
+                    sp.sms = sms;
+                }
+                break;
+            }
+        }
+    }
+    if (nvec > (int64_t)kU * G && sp.cl == 0) {
         // rows longer than one register step of a warp: forward, then the VJP
         // (which re-reads the logits)
         ce_status st = ce_forward(logits, dt, lg, N, V, targets, tdt, tg, label_smoothing,
@@ -413,7 +433,6 @@ ce_status ce_forward_backward(const void* logits, ce_dtype dt, ce_layout lg, int
         if (!in_place && overlap(ed, ez)) return CE_EALIAS;
         if (overlap(ed, et)) return CE_EALIAS;
     }
-    const int sms = device_sms(0);
     FusedPlan p{};
     p.vec = vec;
     p.G = G;
@@ -443,7 +462,9 @@ ce_status ce_forward_backward(const void* logits, ce_dtype dt, ce_layout lg, int
     a.g_stride = grad_stride;
     a.dz = dlogits;
     a.ld = D;
-    cudaError_t e = launch_fused(p, a, (int)dt, (int)ddt, static_cast<cudaStream_t>(cuda_stream));
+    cudaError_t e = sp.cl > 0
+                        ? launch_fused_smem(sp, a, (int)dt, (int)ddt, static_cast<cudaStream_t>(cuda_stream))
+                        : launch_fused(p, a, (int)dt, (int)ddt, static_cast<cudaStream_t>(cuda_stream));
     return e == cudaSuccess ? CE_OK : CE_ECUDA;
 }
 

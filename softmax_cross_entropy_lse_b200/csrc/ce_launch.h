@@ -97,4 +97,19 @@ struct FusedPlan {
 cudaError_t launch_fused(const FusedPlan& p, const FusedArgs& a, int dt_in, int dt_out,
                          cudaStream_t s);
 
+// ---- fused forward + backward (rows held in shared memory) -----------------
+// A row is split over a cluster of `cl` CTAs, vec_per_cta 16-byte vectors
+// each, held in nch 2 KB chunks of shared memory.
+constexpr int kSmemRowMaxChunks = 56;  // 112 KB per CTA: two CTAs per SM
+
+struct SmemRowPlan {
+    int cl;
+    int nch;
+    int64_t vec_per_cta;
+    int sms;
+};
+
+cudaError_t launch_fused_smem(const SmemRowPlan& p, const FusedArgs& a, int dt_in, int dt_out,
+                              cudaStream_t s);
+
 }  // namespace ceb

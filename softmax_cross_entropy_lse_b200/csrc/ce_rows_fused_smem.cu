@@ -1,0 +1,371 @@
+// Fused forward + VJP for rows held in shared memory (rows too long for one
+// warp's registers, up to 8 x 112 KB).
+//
+// When g is known before the forward runs, the gradient
+//     dz_j = g (exp(z_j - lse) - (1 - eps)[j = y] - eps/V)
+// needs nothing but the row and its lse, so the row is read from HBM once:
+// it is copied into shared memory, folded into the online (max, scaled sum)
+// state of Ineshin, "A fused linear cross-entropy forward kernel for Apple
+// GPUs", section 1, reduced, and then read a second time from shared memory
+// to form dz. HBM traffic is 2 V e per row instead of the 3 V e of a forward
+// followed by a VJP that re-reads the logits (the backward regenerates from
+// the saved lse, section 1 of the same page).
+//
+// A row longer than one CTA's share of shared memory is split across a
+// thread-block cluster of CL CTAs (CL = 1, 2, 4, 8); CTA k holds vectors
+// [k S, (k+1) S) of the row. Each CTA reduces its slice, the CL partial
+// states are exchanged once through distributed shared memory, and every CTA
+// merges them in rank order, so all of them derive the same lse bits.
+//
+// Within a CTA, 8 warps own the 2 KB chunks of the slice round-robin (chunk c
+// belongs to warp c % 8). A warp's lane 0 copies its chunks in with 1-D bulk
+// copies (TMA engine), the warp folds them as they land, and after the
+// gradient pass over a chunk it refills that chunk with the next row's bytes
+// at once: no CTA-wide barrier guards the buffers, and the next row streams
+// in while this one is being differentiated. The warp and CTA states of row
+// i use exchange slots of parity i & 1, so no slot is rewritten before every
+// reader has passed the next barrier (the race of Suryavanshi, "One barrier
+// short", cannot occur). Every wait is bounded; on expiry the kernel raises
+// error bit 2, stops issuing copies, drains those in flight and returns.
+#include "ce_device.cuh"
+#include "ce_launch.h"
+#include "ce_sm100.cuh"
+
+#include <atomic>
+
+namespace ceb {
+
+constexpr int kSmWarps = 8;
+constexpr int kSmChunkVecs = 128;  // 16-byte vectors per 2 KB chunk
+constexpr int kSmMaxChunks = kSmemRowMaxChunks;
+static_assert(kSmMaxChunks <= 8 * 32, "per-warp chunk masks are 32 bits");
+
+struct __align__(8) StateRec {
+    float m, s, t;
+    int k;
+    float av;
+    int ai;
+};
+
+template <typename TI, bool ARGMAX, bool WITH_T>
+__device__ __forceinline__ void fold_chunk(OnlineState& st, const uint4* buf, int nvc, int lane,
+                                           int64_t col_vec0) {
+    constexpr int VEC = ElemTraits<TI>::kVec;
+    constexpr int kPerLane = kSmChunkVecs / 32;
+    if constexpr (sizeof(TI) == 2 && !ARGMAX) {
+        uint4 w[kPerLane];
+        bool ok[kPerLane];
+#pragma unroll
+        for (int q = 0; q < kPerLane; ++q) {
+            const int vi = q * 32 + lane;
+            ok[q] = vi < nvc;
+            if (ok[q]) w[q] = buf[vi];
+        }
+        if (nvc == kSmChunkVecs)
+            fold_raw16<TI, kPerLane, false, WITH_T>(st, w, ok);
+        else
+            fold_raw16<TI, kPerLane, true, WITH_T>(st, w, ok);
+    } else {
+        float v[kPerLane][VEC];
+        bool ok[kPerLane];
+        int c0[kPerLane];
+#pragma unroll
+        for (int q = 0; q < kPerLane; ++q) {
+            const int vi = q * 32 + lane;
+            ok[q] = vi < nvc;
+            c0[q] = (int)((col_vec0 + vi) * VEC);
+            if (ok[q]) unpack_words<TI>(buf[vi], v[q]);
+        }
+        if (nvc == kSmChunkVecs) {
+            fold_vecs<kPerLane, VEC, false>(st, v, ok);
+            if constexpr (ARGMAX) argmax_vecs<kPerLane, VEC, false>(st, v, ok, c0);
+        } else {
+            fold_vecs<kPerLane, VEC, true>(st, v, ok);
+            if constexpr (ARGMAX) argmax_vecs<kPerLane, VEC, true>(st, v, ok, c0);
+        }
+    }
+}
+
+// dz of one chunk from its shared-memory copy. `cst` is 0 for ordinary rows;
+// ignored rows write 0 and rows with a bad target NaN (cst_mode 1 / 2).
+template <typename TI, typename TO>
+__device__ __forceinline__ void grad_chunk(const uint4* buf, int nvc, int lane, int64_t col_vec0,
+                                           TO* drow, float hi, float c_lo, float g, float c_eps,
+                                           float c_tgt, int64_t yc, int cst_mode) {
+    constexpr int VEC = ElemTraits<TI>::kVec;
+    constexpr int kPerLane = kSmChunkVecs / 32;
+    const int64_t col_chunk = col_vec0 * VEC;
+    const bool has_y = yc >= col_chunk && yc < col_chunk + (int64_t)nvc * VEC;
+    const float2 nhi = make_float2(-hi, -hi), l2 = make_float2(kLog2e, kLog2e);
+    const float2 nclo = make_float2(-c_lo, -c_lo), g2 = make_float2(g, g);
+    const float2 nce = make_float2(-c_eps, -c_eps);
+    const float fill = cst_mode == 2 ? __int_as_float(0x7fc00000) : 0.f;
+#pragma unroll
+    for (int q = 0; q < kPerLane; ++q) {
+        const int vi = q * 32 + lane;
+        if (vi >= nvc) continue;
+        const int64_t col0 = (col_vec0 + vi) * VEC;
+        float o[VEC];
+        if (cst_mode != 0) {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) o[e] = fill;
+        } else {
+            float x[VEC];
+            unpack_words<TI>(buf[vi], x);
+#pragma unroll
+            for (int e = 0; e < VEC; e += 2) {
+                const float2 d = __fadd2_rn(make_float2(x[e], x[e + 1]), nhi);
+                const float2 arg = __ffma2_rn(d, l2, nclo);
+                const float2 p = make_float2(ex2(arg.x), ex2(arg.y));
+                const float2 r = __ffma2_rn(g2, p, nce);
+                o[e] = r.x;
+                o[e + 1] = r.y;
+            }
+            if (has_y) {
+                const int64_t dy = yc - col0;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e)
+                    if (dy == e) o[e] -= c_tgt;
+            }
+        }
+        store_vec<TO, VEC>(drow, col0, 1, o);
+    }
+}
+
+template <typename TI, typename TO, int CL, bool ARGMAX, bool WITH_T>
+__global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, SmemRowPlan sp) {
+    using namespace sm100;
+    constexpr int VEC = ElemTraits<TI>::kVec;
+    const FwdArgs& a = fa.f;
+    extern __shared__ __align__(128) uint8_t row_smem[];
+    __shared__ __align__(8) uint64_t full_bar[kSmMaxChunks];
+    __shared__ OnlineState wslot[2][kSmWarps];
+    __shared__ StateRec cslot[2];
+    __shared__ int abort_flag;
+
+    const TI* z = reinterpret_cast<const TI*>(a.z);
+    TO* dz = reinterpret_cast<TO*>(fa.dz);
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const uint32_t rank = CL == 1 ? 0u : cluster_ctarank();
+    const int64_t cid = CL == 1 ? (int64_t)blockIdx.x : (int64_t)cluster_id_x();
+    const int64_t ncl = CL == 1 ? (int64_t)gridDim.x : (int64_t)cluster_count_x();
+    const int64_t nvec = a.V / VEC;
+    const int tail = (int)(a.V - nvec * VEC);
+    const int64_t v0 = (int64_t)rank * sp.vec_per_cta;
+    const int64_t v1 = min(nvec, v0 + sp.vec_per_cta);
+    const int nv = v1 > v0 ? (int)(v1 - v0) : 0;
+    const int nch = (nv + kSmChunkVecs - 1) / kSmChunkVecs;
+    const bool tail_here = rank == CL - 1 && wid == 0 && tail > 0;
+    const RowOut out{a.loss, a.lse, a.lse_lo, a.argmax, a.err};
+    const float inv_v = 1.f / (float)a.V;
+
+    if (lane == 0)
+        for (int c = wid; c < nch; c += kSmWarps) mbar_init(smem_u32(&full_bar[c]), 1);
+    if (tid == 0) abort_flag = 0;
+    if (lane == 0) mbar_fence_init();
+    __syncthreads();
+
+    auto chunk_vecs = [&](int c) { return min(kSmChunkVecs, nv - c * kSmChunkVecs); };
+    auto chunk_buf = [&](int c) { return reinterpret_cast<const uint4*>(row_smem + (size_t)c * 2048); };
+    auto issue = [&](int64_t r, int c) {
+        const uint32_t bar = smem_u32(&full_bar[c]);
+        const uint32_t bytes = (uint32_t)chunk_vecs(c) * 16u;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(z + row_offset(a.lz, r, a.N)) +
+                             (v0 + (int64_t)c * kSmChunkVecs) * 16;
+        mbar_expect_tx(bar, bytes);
+        bulk_load(smem_u32(row_smem + (size_t)c * 2048), src, bytes, bar);
+    };
+
+    // bit i of the masks: this warp's i-th chunk (c = wid + 8 i)
+    uint32_t pend = 0, phase = 0;
+    if (cid < a.N) {
+        for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps) {
+            if (lane == 0) issue(cid, c);
+            pend |= 1u << i;
+        }
+    }
+
+    bool dead = false;
+    int it = 0;
+    for (int64_t r = cid; r < a.N; r += ncl, ++it) {
+        const int par = it & 1;
+        const TI* row = z + row_offset(a.lz, r, a.N);
+        TO* drow = dz + row_offset(fa.ld, r, a.N);
+        const int64_t y = load_target(a.y, a.tdt, row_offset(a.ly, r, a.N));
+        const float g = fa.g[r * fa.g_stride];
+        const bool ign = y == a.ignore;
+        const bool bad = !ign && (y < 0 || y >= a.V);
+        const int64_t yc = (ign || bad) ? -1 : y;
+        float zy = 0.f;
+        if (rank == 0 && tid == 0 && yc >= 0) zy = to_f32(row[yc]);
+
+        // ---- forward: fold the slice as its chunks land
+        OnlineState st = empty_state();
+        for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps) {
+            if (!dead) {
+                if (mbar_wait(smem_u32(&full_bar[c]), (phase >> i) & 1u, &abort_flag)) {
+                    phase ^= 1u << i;
+                    pend &= ~(1u << i);
+                } else {
+                    dead = true;
+                }
+            }
+            if (!dead)
+                fold_chunk<TI, ARGMAX, WITH_T>(st, chunk_buf(c), chunk_vecs(c), lane,
+                                               v0 + (int64_t)c * kSmChunkVecs);
+        }
+        if (tail_here) {
+            for (int q = lane; q < tail; q += 32) {
+                float x;
+                load_vec_coherent<TI, 1>(row, nvec * VEC + q, 1, &x);
+                fold<1, ARGMAX>(st, &x, (int)(nvec * VEC + q), 0);
+            }
+        }
+        group_reduce<32, ARGMAX>(st);
+        if (lane == 0) wslot[par][wid] = st;
+        __syncthreads();
+        // every warp merges the 8 warp states in the same order (same bits)
+        st = wslot[par][lane & (kSmWarps - 1)];
+        group_reduce<kSmWarps, ARGMAX>(st);
+        if constexpr (CL > 1) {
+            if (tid == 0) {
+                StateRec rec{st.m, st.s, st.t, st.k, st.av, st.ai};
+                cslot[par] = rec;
+            }
+            cluster_sync();
+            const uint32_t ra = mapa_shared(smem_u32(&cslot[par]), (uint32_t)(lane & (CL - 1)));
+            const uint2 p0 = ld_cluster_v2(ra), p1 = ld_cluster_v2(ra + 8), p2 = ld_cluster_v2(ra + 16);
+            st.m = __uint_as_float(p0.x);
+            st.s = __uint_as_float(p0.y);
+            st.t = __uint_as_float(p1.x);
+            st.k = (int)p1.y;
+            st.av = __uint_as_float(p2.x);
+            st.ai = (int)p2.y;
+            group_reduce<CL, ARGMAX>(st);
+        }
+        if (rank == 0 && tid == 0) finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);
+
+        // ---- backward from the same shared-memory copy
+        float L, hi, lo;
+        lse_pair(st, L, hi, lo);
+        const float c_lo = lo * kLog2e, c_eps = g * a.eps * inv_v, c_tgt = g * (1.f - a.eps);
+        const int cst_mode = bad ? 2 : (ign ? 1 : 0);
+        const int64_t rn = r + ncl;
+        for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps) {
+            if (!dead)
+                grad_chunk<TI, TO>(chunk_buf(c), chunk_vecs(c), lane, v0 + (int64_t)c * kSmChunkVecs,
+                                   drow, hi, c_lo, g, c_eps, c_tgt, yc, cst_mode);
+            // the chunk is read: refill it with the next row's bytes
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (rn < a.N && !dead) {
+                if (lane == 0) issue(rn, c);
+                pend |= 1u << i;
+            }
+        }
+        if (tail_here) {
+            for (int q = lane; q < tail; q += 32) {
+                const int64_t col = nvec * VEC + q;
+                float d;
+                if (cst_mode != 0) {
+                    d = cst_mode == 2 ? __int_as_float(0x7fc00000) : 0.f;
+                } else {
+                    float x;
+                    load_vec_coherent<TI, 1>(row, col, 1, &x);
+                    d = fmaf(g, ex2(fmaf(x - hi, kLog2e, -c_lo)), -c_eps);
+                    if (col == yc) d -= c_tgt;
+                }
+                cvt_store1(drow + col, d);
+            }
+        }
+    }
+
+    if (dead || abort_flag) {
+        if (lane == 0) atomicOr(a.err, 2u);
+        // let every copy this warp started land before the CTA exits
+        volatile int never = 0;
+        for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps)
+            if ((pend >> i) & 1u) mbar_wait(smem_u32(&full_bar[c]), (phase >> i) & 1u, &never);
+    }
+    // no CTA leaves while another may still read its exchange slot
+    if constexpr (CL > 1) cluster_sync();
+}
+
+// ---------------------------------------------------------------------------
+template <typename TI, typename TO, int CL, bool ARGMAX, bool WITH_T>
+static cudaError_t launch_smem_k(const SmemRowPlan& sp, const FusedArgs& a, cudaStream_t s) {
+    auto kern = k_fwdbwd_smem<TI, TO, CL, ARGMAX, WITH_T>;
+    static std::atomic<int> attr{0};
+    if (!attr.load(std::memory_order_relaxed)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kSmMaxChunks * 2048);
+        if (e != cudaSuccess) return e;
+        attr.store(1, std::memory_order_relaxed);
+    }
+    const size_t smem = (size_t)sp.nch * 2048;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    cfg.blockDim = dim3(kSmWarps * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = CL;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = CL > 1 ? 1 : 0;
+    // co-resident clusters (CTAs when CL = 1) for this shared-memory size,
+    // cached per size
+    static std::atomic<long long> cached{0};  // (smem << 20) | clusters
+    const long long c = cached.load(std::memory_order_relaxed);
+    int clusters = 0;
+    if (c != 0 && (size_t)(c >> 20) == smem) {
+        clusters = (int)(c & 0xfffff);
+    } else {
+        cudaError_t e;
+        if constexpr (CL > 1) {
+            cfg.gridDim = dim3(CL * sp.sms);
+            e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+        } else {
+            int per_sm = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSmWarps * 32, smem);
+            clusters = per_sm * sp.sms;
+        }
+        if (e != cudaSuccess) return e;
+        if (clusters < 1) return cudaErrorInvalidConfiguration;
+        cached.store(((long long)smem << 20) | clusters, std::memory_order_relaxed);
+    }
+    const int64_t want = a.f.N < clusters ? a.f.N : clusters;
+    cfg.gridDim = dim3((unsigned)(want * CL));
+    return cudaLaunchKernelEx(&cfg, kern, a, sp);
+}
+
+template <typename TI, typename TO, bool ARGMAX, bool WITH_T>
+static cudaError_t launch_smem_cl(const SmemRowPlan& sp, const FusedArgs& a, cudaStream_t s) {
+    switch (sp.cl) {
+        case 1: return launch_smem_k<TI, TO, 1, ARGMAX, WITH_T>(sp, a, s);
+        case 2: return launch_smem_k<TI, TO, 2, ARGMAX, WITH_T>(sp, a, s);
+        case 4: return launch_smem_k<TI, TO, 4, ARGMAX, WITH_T>(sp, a, s);
+        case 8: return launch_smem_k<TI, TO, 8, ARGMAX, WITH_T>(sp, a, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+template <typename TI, typename TO>
+static cudaError_t launch_smem_t(const SmemRowPlan& sp, const FusedArgs& a, cudaStream_t s) {
+    const bool am = a.f.argmax != nullptr, t = a.f.eps != 0.f;
+    if (am) return t ? launch_smem_cl<TI, TO, true, true>(sp, a, s) : launch_smem_cl<TI, TO, true, false>(sp, a, s);
+    return t ? launch_smem_cl<TI, TO, false, true>(sp, a, s) : launch_smem_cl<TI, TO, false, false>(sp, a, s);
+}
+
+cudaError_t launch_fused_smem(const SmemRowPlan& sp, const FusedArgs& a, int dt_in, int dt_out,
+                              cudaStream_t s) {
+    if (dt_in == 0 && dt_out == 0) return launch_smem_t<float, float>(sp, a, s);
+    if (dt_in == 1 && dt_out == 1) return launch_smem_t<__nv_bfloat16, __nv_bfloat16>(sp, a, s);
+    if (dt_in == 1 && dt_out == 0) return launch_smem_t<__nv_bfloat16, float>(sp, a, s);
+    if (dt_in == 2 && dt_out == 2) return launch_smem_t<__half, __half>(sp, a, s);
+    if (dt_in == 2 && dt_out == 0) return launch_smem_t<__half, float>(sp, a, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace ceb

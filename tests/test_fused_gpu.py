@@ -132,3 +132,111 @@ def test_bad_targets_and_nonfinite(orc):
     torch.cuda.synchronize()
     assert ce.get_error() == 5
     check_oracle(orc, rf, dzf, z.astype(np.float64), y, 1.0, 0.1, -100, "f32", "f32")
+
+
+# -- rows held in shared memory (one CTA, or a cluster of 2, 4 or 8 per row) ----------------
+def _padded(N, V, pad, dtype, seed, std=2.0, ignore_frac=0.1):
+    """Logits (N, V) as a view of an (N, V + pad) buffer, so rows stay 16-byte
+    aligned when V is not a multiple of the vector width (a ragged tail)."""
+    z, z32, y = wl.rows(N, V + pad, dtype, seed=seed, std=std, ignore_frac=ignore_frac)
+    y = np.where(y >= V, y % V, y).astype(y.dtype)  # targets inside the view
+    return z, z32[:, :V], y
+
+
+@pytest.mark.parametrize("V,N,dt", [
+    (2048, 400, "bf16"),       # one CTA, 2 chunks
+    (32000, 600, "bf16"),      # one CTA, the 8192 x 32000 row shape
+    (33000, 300, "f16"),       # one CTA, partial last chunk
+    (100000, 200, "bf16"),     # cluster of 2
+    (151936, 160, "bf16"),     # cluster of 4, the 2048 x 151,936 row shape
+    (20000, 300, "f32"),       # one CTA, fp32
+    (151936, 40, "f32"),       # cluster of 8, fp32
+])
+def test_smem_rows_vs_oracle(orc, V, N, dt):
+    z, z32, y = wl.rows(N, V, dt, seed=V % 997 + N, std=2.0, ignore_frac=0.1)
+    gv = np.random.default_rng(V).standard_normal(N).astype(np.float32)
+    zt, yt, gt = upload(z, dt), upload(y), upload(gv)
+    for eps, am in ((0.0, False), (0.1, True)):
+        rf, dzf = ce.ce_forward_backward(zt, yt, gt, eps, return_argmax=am)
+        torch.cuda.synchronize()
+        assert ce.get_error() == 0
+        loss, lse, amx = orc.ce_forward(z32.astype(np.float64), y, eps)
+        rt, at = loss_tol(dt)
+        assert_close(f32(rf.loss), loss, rt, at, "loss")
+        assert_close(f32(rf.lse), lse, rt, at, "lse")
+        if am:
+            np.testing.assert_array_equal(rf.argmax.cpu().numpy(), amx)
+        ref = orc.ce_backward(z32.astype(np.float64), y, gv.astype(np.float64), eps)
+        assert_grad_close(f32(dzf), ref, dt, dt)
+        # the same lse as the separate forward, up to the order of the sum
+        rs = ce.ce_forward(zt, yt, eps)
+        assert_close(f32(rf.lse), f32(rs.lse).astype(np.float64), 2e-6, 0.0, "lse vs ce_forward")
+
+
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_smem_rows_ragged_tail_views(orc, out):
+    """V = 32005 (5 columns past the last 16-byte vector), rows of a padded
+    buffer; dlogits is a padded view too, in bf16 or float."""
+    N, V, pad = 300, 32005, 3
+    z, z32, y = _padded(N, V, pad, "bf16", seed=5)
+    zt = upload(z, "bf16")[:, :V]
+    yt = upload(y)
+    od = torch.bfloat16 if out == "bf16" else torch.float32
+    dbuf = torch.empty((N, V + pad), dtype=od, device="cuda")
+    dv = dbuf[:, :V]
+    rf, dzf = ce.ce_forward_backward(zt, yt, torch.ones(1, device="cuda"), 0.2,
+                                     return_argmax=True, dlogits=dv)
+    torch.cuda.synchronize()
+    assert dzf.data_ptr() == dbuf.data_ptr()
+    check_oracle(orc, rf, dzf, z32.astype(np.float64), y, 1.0, 0.2, -100, "bf16", out)
+
+
+def test_smem_rows_strided_3d_view_cluster(orc):
+    """The (B, L, V) view x[:, :-1] at V = 151,936 fp32 (rows of 607,744 bytes,
+    a cluster of 8 CTAs per row), targets t[:, 1:]."""
+    x, t = wl.c4a(B=3, L=21, V=151936)
+    xt, tt = upload(x), upload(t)
+    zv, yv = xt[:, :-1], tt[:, 1:]
+    g = torch.full((1,), 0.5, device="cuda")
+    rf, dzf = ce.ce_forward_backward(zv, yv, g, 0.0, return_argmax=True, dlogits=zv.clone())
+    torch.cuda.synchronize()
+    z64 = x[:, :-1].reshape(-1, x.shape[-1]).astype(np.float64)
+    y = t[:, 1:].reshape(-1)
+    check_oracle(orc, rf, dzf.reshape(-1, x.shape[-1]), z64, y, 0.5, 0.0, -100, "f32", "f32")
+
+
+def test_smem_rows_in_place_and_repeatable():
+    z, z32, y = wl.rows(300, 32000, "bf16", seed=9, std=2.0, ignore_frac=0.2)
+    zt, yt = upload(z, "bf16"), upload(y)
+    g = torch.ones(1, device="cuda")
+    r1, d1 = ce.ce_forward_backward(zt, yt, g, 0.1, return_argmax=True)
+    r2, d2 = ce.ce_forward_backward(zt, yt, g, 0.1, return_argmax=True)
+    zc = zt.clone()
+    r3, d3 = ce.ce_forward_backward(zc, yt, g, 0.1, return_argmax=True, dlogits=zc)
+    torch.cuda.synchronize()
+    for a, b in zip(r1, r2):
+        assert torch.equal(a, b)
+    assert torch.equal(d1, d2)
+    for a, b in zip(r1, r3):
+        assert torch.equal(a, b)
+    assert d3.data_ptr() == zc.data_ptr() and torch.equal(d1, zc)
+
+
+def test_smem_rows_bad_targets_and_nonfinite(orc):
+    N, V = 200, 40000
+    rng = np.random.default_rng(7)
+    z32 = rng.standard_normal((N, V)).astype(np.float32)
+    y = rng.integers(0, V, size=N).astype(np.int32)
+    y[3] = V
+    y[4] = -7
+    y[5] = -100
+    z32[6, 12345] = np.nan
+    z32[7, :] = -np.inf
+    z32[8, 100:200] = -np.inf
+    z32[9, y[9]] = -np.inf
+    z32[10, :] = 1e30
+    rf, dzf = ce.ce_forward_backward(upload(z32), upload(y), torch.ones(1, device="cuda"), 0.0,
+                                     return_argmax=True)
+    torch.cuda.synchronize()
+    assert ce.get_error() == 5
+    check_oracle(orc, rf, dzf, z32.astype(np.float64), y, 1.0, 0.0, -100, "f32", "f32")
