@@ -134,6 +134,18 @@ static FwdPlan plan_forward(int64_t N, int64_t V, int esz, bool vec_ok, int sms)
     p.vec = vec_ok ? vecw : 1;
     p.splits = 1;
     p.vec_per_split = 0;
+    if (vec_ok && V % vecw == 0 && V / vecw <= 2) {
+        // one or two whole vectors per row: a lane per row
+        p.kind = FwdPlan::kTiny;
+        p.G = 1;
+        p.U = (int)(V / vecw);
+        p.R = kTinyRows;
+        const int64_t rows_per_block = 256 * (int64_t)kTinyRows;
+        const int64_t want = (N + rows_per_block - 1) / rows_per_block;
+        const int64_t cap = (int64_t)sms * (p.U == 1 ? 5 : 4);  // every block resident
+        p.grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
+        return p;
+    }
     if (use_packed(V, esz) || (!vec_ok && V <= 256)) {
         p.kind = FwdPlan::kPacked;
         const int64_t nvec = V / p.vec;

@@ -195,10 +195,14 @@ __device__ __forceinline__ bool argmax_better(float bv, int bi, float av, int ai
 }
 
 // Rescale the state to a new max mn >= st.m (st.m = -inf gives factor 0).
+// Without WITH_T the state carries only (m, s): t and k are left untouched.
+template <bool WITH_T = true>
 __device__ __forceinline__ void rescale_to(OnlineState& st, float mn) {
     if (st.m != mn) {
         st.s *= ex2((st.m - mn) * kLog2e);
-        if (st.k != 0) st.t += (float)st.k * (st.m - mn);
+        if constexpr (WITH_T) {
+            if (st.k != 0) st.t += (float)st.k * (st.m - mn);
+        }
         st.m = mn;
     }
 }
@@ -348,7 +352,7 @@ __device__ __forceinline__ void fold_raw16(OnlineState& st, const uint4 (&w)[U],
         mx = R::max2(mx, R::max2(R::max2(w[u].x, w[u].y), R::max2(w[u].z, w[u].w)));
     }
     const float2 m2 = R::widen(mx);
-    rescale_to(st, fmaxf(st.m, fmaxf(m2.x, m2.y)));
+    rescale_to<WITH_T>(st, fmaxf(st.m, fmaxf(m2.x, m2.y)));
     const float ms = (st.m == -INFINITY) ? 0.f : st.m;
     const float2 l2 = make_float2(kLog2e, kLog2e);
     const float2 nm = make_float2(-ms, -ms);
@@ -371,8 +375,10 @@ __device__ __forceinline__ void fold_raw16(OnlineState& st, const uint4 (&w)[U],
         n += 8;
     }
     st.s += sa.x + sa.y;
-    if constexpr (WITH_T) st.t += ta.x + ta.y;
-    st.k += n;
+    if constexpr (WITH_T) {
+        st.t += ta.x + ta.y;
+        st.k += n;
+    }
 }
 
 // Argmax over U vectors whose first columns are col0[u], in increasing
@@ -431,15 +437,49 @@ __device__ __forceinline__ OnlineState shfl_xor_state(const OnlineState& st, int
     return o;
 }
 
-// Butterfly over groups of G lanes (G a power of two <= 32). Every lane of the
-// warp must call it. Addition and multiplication commute exactly, so every
-// lane of a group ends with the same bits.
-template <int G, bool ARGMAX>
+// Reduction over groups of G lanes (G a power of two <= 32). Every lane of
+// the warp must call it. Addition and multiplication commute exactly, so
+// every lane of a group ends with the same bits.
+//
+// With argmax, states are merged pairwise along a butterfly. Without, the
+// group takes its max first, every lane rescales its own (s, t) to it once,
+// and the rescaled terms are summed along the butterfly: the same merge
+// operator, with one exponential per lane instead of two per round. WITH_T =
+// false reduces (m, s) only (t and k are left as they are).
+template <int G, bool ARGMAX, bool WITH_T = true>
 __device__ __forceinline__ void group_reduce(OnlineState& st) {
+    if constexpr (ARGMAX) {
 #pragma unroll
-    for (int off = G / 2; off >= 1; off >>= 1) {
-        OnlineState o = shfl_xor_state<ARGMAX>(st, off);
-        merge<ARGMAX>(st, o);
+        for (int off = G / 2; off >= 1; off >>= 1) {
+            OnlineState o = shfl_xor_state<ARGMAX>(st, off);
+            merge<ARGMAX>(st, o);
+        }
+    } else if constexpr (G > 1) {
+        float M = st.m;
+#pragma unroll
+        for (int off = G / 2; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        float s = st.s, t = st.t;
+        int k = st.k;
+        if (st.m != M) {
+            s *= ex2((st.m - M) * kLog2e);
+            if constexpr (WITH_T) {
+                if (k != 0) t += (float)k * (st.m - M);
+            }
+        }
+#pragma unroll
+        for (int off = G / 2; off >= 1; off >>= 1) {
+            s += __shfl_xor_sync(0xffffffffu, s, off);
+            if constexpr (WITH_T) {
+                t += __shfl_xor_sync(0xffffffffu, t, off);
+                k += __shfl_xor_sync(0xffffffffu, k, off);
+            }
+        }
+        st.m = M;
+        st.s = s;
+        if constexpr (WITH_T) {
+            st.t = t;
+            st.k = k;
+        }
     }
 }
 

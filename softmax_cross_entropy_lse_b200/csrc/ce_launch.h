@@ -34,9 +34,9 @@ struct FwdArgs {
 };
 
 struct FwdPlan {
-    enum Kind { kPacked = 0, kCta = 1 } kind;
+    enum Kind { kPacked = 0, kCta = 1, kTiny = 2 } kind;
     int vec;        // 1 (scalar path) or the 16-byte vector width of the dtype
-    int G, U;       // packed: lanes per row, vectors per lane per step
+    int G, U;       // packed: lanes per row, vectors per lane per step; tiny: U vectors per row
     int R;          // packed: rows per group per step
     int ring;       // long rows through per-warp bulk-copy rings
     int grid;
@@ -46,6 +46,9 @@ struct FwdPlan {
 };
 
 cudaError_t launch_forward(const FwdPlan& p, const FwdArgs& a, int dtype, cudaStream_t s);
+
+// rows per lane per step of the tiny-row forward
+constexpr int kTinyRows = 2;
 int cta_threads_forward();
 
 // ---- row backward ------------------------------------------------------------

@@ -221,12 +221,12 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
                 fold<1, ARGMAX>(st, &x, (int)(nvec * VEC + q), 0);
             }
         }
-        group_reduce<32, ARGMAX>(st);
+        group_reduce<32, ARGMAX, WITH_T>(st);
         if (lane == 0) wslot[par][wid] = st;
         __syncthreads();
         // every warp merges the 8 warp states in the same order (same bits)
         st = wslot[par][lane & (kSmWarps - 1)];
-        group_reduce<kSmWarps, ARGMAX>(st);
+        group_reduce<kSmWarps, ARGMAX, WITH_T>(st);
         if constexpr (CL > 1) {
             if (tid == 0) {
                 StateRec rec{st.m, st.s, st.t, st.k, st.av, st.ai};
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
             st.k = (int)p1.y;
             st.av = __uint_as_float(p2.x);
             st.ai = (int)p2.y;
-            group_reduce<CL, ARGMAX>(st);
+            group_reduce<CL, ARGMAX, WITH_T>(st);
         }
         if (rank == 0 && tid == 0) finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);
 

@@ -100,6 +100,107 @@ __global__ void __launch_bounds__(256, MINB) k_fwd_packed(FwdArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Tiny rows: one or two 16-byte vectors and no ragged tail (for instance 8
+// floats). One lane per row and R rows per lane per step, with every load of
+// the step issued before any is used. The whole row sits in registers, so it
+// is folded in one piece: its max first (three-operand max instructions),
+// then the sum of exponentials, with no running state to rescale. z_y is
+// picked from the registers by a select tree on the bits of the target.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+template <int n>
+__device__ __forceinline__ float select_tree(const float (&x)[n], int idx) {
+    static_assert((n & (n - 1)) == 0, "power of two");
+    float v[n];
+#pragma unroll
+    for (int i = 0; i < n; ++i) v[i] = x[i];
+#pragma unroll
+    for (int w = n / 2, b = 1; w >= 1; w >>= 1, b <<= 1) {
+        const bool hi = (idx & b) != 0;
+#pragma unroll
+        for (int i = 0; i < w; ++i) v[i] = hi ? v[2 * i + 1] : v[2 * i];
+    }
+    return v[0];
+}
+
+template <typename T, int VEC, int NV, int R, bool ARGMAX, bool WITH_T, int MINB>
+__global__ void __launch_bounds__(256, MINB) k_fwd_tiny(FwdArgs a) {
+    constexpr int n = NV * VEC;
+    const T* __restrict__ z = reinterpret_cast<const T*>(a.z);
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const RowOut out{a.loss, a.lse, a.lse_lo, a.argmax, a.err};
+
+    for (int64_t base = warp * 32 * R; base < a.N; base += nwarps * 32 * R) {
+        uint4 w[R][NV];
+        int64_t y[R];
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            const int64_t r = base + 32 * k + lane;
+            y[k] = a.ignore;
+            if (r < a.N) {
+                const T* row = z + row_offset(a.lz, r, a.N);
+                y[k] = load_target(a.y, a.tdt, row_offset(a.ly, r, a.N));
+#pragma unroll
+                for (int v = 0; v < NV; ++v) w[k][v] = __ldcs(reinterpret_cast<const uint4*>(row) + v);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            const int64_t r = base + 32 * k + lane;
+            if (r >= a.N) continue;
+            float x[n];
+#pragma unroll
+            for (int v = 0; v < NV; ++v) unpack_words<T>(w[k][v], x + v * VEC);
+            float m = fmaxf(x[0], x[1]);
+#pragma unroll
+            for (int i = 2; i + 1 < n; i += 2) m = fmax3(m, x[i], x[i + 1]);
+            OnlineState st = empty_state();
+            st.m = m;
+            const float ms = m == -INFINITY ? 0.f : m;
+            const float2 nm = make_float2(-ms, -ms), l2 = make_float2(kLog2e, kLog2e);
+            // per-vector partial pairs, then across vectors: the order of
+            // fold_vecs, so the fused forward + VJP gets the same bits
+            float2 sa = make_float2(0.f, 0.f), ta = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int v = 0; v < NV; ++v) {
+                float2 su = make_float2(0.f, 0.f), tu = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int i = v * VEC; i < (v + 1) * VEC; i += 2) {
+                    const float2 d = __fadd2_rn(make_float2(x[i], x[i + 1]), nm);
+                    const float2 d2 = __fmul2_rn(d, l2);
+                    su = __fadd2_rn(su, make_float2(ex2(d2.x), ex2(d2.y)));
+                    if constexpr (WITH_T) tu = __fadd2_rn(tu, d);
+                }
+                sa = __fadd2_rn(sa, su);
+                if constexpr (WITH_T) ta = __fadd2_rn(ta, tu);
+            }
+            st.s = sa.x + sa.y;
+            st.t = ta.x + ta.y;
+            st.k = n;
+            if constexpr (ARGMAX) {
+#pragma unroll
+                for (int i = 0; i < n; ++i) {
+                    const float xi = x[i];
+                    if ((st.ai < 0) | (xi > st.av) | ((xi != xi) & (st.av == st.av))) {
+                        st.av = xi;
+                        st.ai = i;
+                    }
+                }
+            }
+            const int64_t yk = y[k];
+            const float zy = select_tree<n>(x, (int)(yk & (n - 1)));
+            finalize_row(st, zy, yk, a.ignore, a.V, a.eps, out, r, ARGMAX);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // CTA rows. Unit u = (row, split) with split-major order inside a row.
 constexpr int kCtaThreads = 512;
 constexpr int kCtaMinBlocks = 2;
@@ -170,8 +271,8 @@ __global__ void __launch_bounds__(kCtaThreads, kCtaMinBlocks) k_fwd_cta(FwdArgs 
         if (lane == 0) slots[parity][wid] = st;
         __syncthreads();
         if (wid == 0) {
-            st = lane < kCtaWarps ? slots[parity][lane] : empty_state();
-            group_reduce<32, ARGMAX>(st);
+            st = slots[parity][lane & (kCtaWarps - 1)];
+            group_reduce<kCtaWarps, ARGMAX>(st);
             if (lane == 0) {
                 if (a.splits == 1) {
                     finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);
@@ -203,6 +304,8 @@ constexpr int kRingWarps = 8;
 constexpr int kRingStages = 4;
 constexpr int kRingVecs = 128;  // 2 KB per stage
 constexpr size_t kRingSmem = (size_t)kRingWarps * kRingStages * kRingVecs * 16;
+static_assert((kRingStages & (kRingStages - 1)) == 0 && (kRingWarps & (kRingWarps - 1)) == 0,
+              "stage and warp counts are powers of two");
 
 struct RingUnit {
     const uint8_t* src;  // first byte of the unit's vectors
@@ -284,7 +387,9 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
     // prologue: the first kRingStages chunks of this warp's sequence
     RingCursor<T> iss;
     iss.start(a, units, nvec, wid);
-    int64_t issued = 0;
+    // 32-bit counters: stage = count % 4 and parity = (count / 4) % 2 stay
+    // exact across wraparound (4 and 8 divide 2^32)
+    uint32_t issued = 0;
     for (int q = 0; q < kRingStages && iss.valid(units); ++q) {
         if (lane == 0) {
             const uint32_t bar = smem_u32(&full_bar[wid][q]);
@@ -295,7 +400,7 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
         iss.next(a, units, nvec, wid);
     }
 
-    int64_t consumed = 0, waited = 0;
+    uint32_t consumed = 0, waited = 0;
     bool dead = false;
     int parity = 0;
     for (int64_t u = blockIdx.x; u < units; u += gridDim.x, parity ^= 1) {
@@ -311,10 +416,10 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
         }
         OnlineState st = empty_state();
         for (int j = wid; j < ru.nch; j += kRingWarps) {
-            const int stage = (int)(consumed % kRingStages);
+            const int stage = (int)(consumed & (kRingStages - 1));
             const uint32_t bar = smem_u32(&full_bar[wid][stage]);
             if (!dead) {
-                if (mbar_wait(bar, (uint32_t)((consumed / kRingStages) & 1), &abort_flag))
+                if (mbar_wait(bar, (consumed / kRingStages) & 1u, &abort_flag))
                     ++waited;
                 else
                     dead = true;
@@ -377,12 +482,12 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
                 fold<1, ARGMAX>(st, &x, (int)(nvec * VEC + q), 0);
             }
         }
-        group_reduce<32, ARGMAX>(st);
+        group_reduce<32, ARGMAX, WITH_T>(st);
         if (lane == 0) slots[parity][wid] = st;
         __syncthreads();
         if (wid == 0) {
-            st = lane < kRingWarps ? slots[parity][lane] : empty_state();
-            group_reduce<32, ARGMAX>(st);
+            st = slots[parity][lane & (kRingWarps - 1)];
+            group_reduce<kRingWarps, ARGMAX, WITH_T>(st);
             if (lane == 0) {
                 if (a.splits == 1) {
                     finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);
@@ -403,8 +508,8 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
         // let every copy this warp started land before the CTA exits
         if (lane == 0) {
             volatile int never = 0;
-            for (int64_t e = waited; e < issued; ++e)
-                mbar_wait(smem_u32(&full_bar[wid][e % kRingStages]), (uint32_t)((e / kRingStages) & 1),
+            for (uint32_t e = waited; e != issued; ++e)
+                mbar_wait(smem_u32(&full_bar[wid][e & (kRingStages - 1)]), (e / kRingStages) & 1u,
                           &never);
         }
     }
@@ -484,9 +589,22 @@ static cudaError_t launch_ring(const FwdPlan& p, const FwdArgs& a, cudaStream_t 
     return cudaGetLastError();
 }
 
+template <typename T, bool ARGMAX, bool WITH_T>
+static cudaError_t launch_tiny(const FwdPlan& p, const FwdArgs& a, cudaStream_t s) {
+    constexpr int V8 = ElemTraits<T>::kVec;
+    // register budgets: 51 per thread for one vector per row, 64 for two
+    if (p.U == 1)
+        k_fwd_tiny<T, V8, 1, kTinyRows, ARGMAX, WITH_T, 5><<<p.grid, 256, 0, s>>>(a);
+    else
+        k_fwd_tiny<T, V8, 2, kTinyRows, ARGMAX, WITH_T, 4><<<p.grid, 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
 template <typename T, bool ARGMAX>
 static cudaError_t launch_fwd_t(const FwdPlan& p, const FwdArgs& a, cudaStream_t s) {
     constexpr int V8 = ElemTraits<T>::kVec;
+    if (p.kind == FwdPlan::kTiny)
+        return a.eps != 0.f ? launch_tiny<T, ARGMAX, true>(p, a, s) : launch_tiny<T, ARGMAX, false>(p, a, s);
     if (p.kind == FwdPlan::kPacked) {
         return p.vec == 1 ? launch_packed<T, 1, ARGMAX>(a, p.G, p.U, p.grid, s)
                           : launch_packed<T, V8, ARGMAX>(a, p.G, p.U, p.grid, s);

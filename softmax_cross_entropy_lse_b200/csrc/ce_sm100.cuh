@@ -68,14 +68,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended (issuing nothing) for up
+// to `hint_ns` nanoseconds while the phase is incomplete; it resumes as soon
+// as the phase completes. Waiting warps then leave the issue slots to the
+// warps that have work.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity,
+                                                      uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+constexpr uint32_t kSuspendHintNs = 20000;
+
 // Waits for the phase of parity `parity` to complete. Returns false (and
 // raises *abort) when the time limit passes or another role already aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0) {
+        if (mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) return true;
+        if ((i & 15u) == 0) {
             if (*abort) return false;
             if (globaltimer() - t0 > kWaitTimeoutNs) {
                 *abort = 1;

@@ -111,7 +111,8 @@ def test_in_place_and_strided(orc):
     zv, yv = xt[:, :-1], tt[:, 1:]
     ref_r, ref_dz = separate(zv, yv, torch.ones(1, device="cuda"), 0.0)
     ref_dz = ref_dz.clone()
-    rf, dzf = ce.ce_forward_backward(zv, yv, torch.ones(1, device="cuda"), dlogits=zv)
+    rf, dzf = ce.ce_forward_backward(zv, yv, torch.ones(1, device="cuda"), dlogits=zv,
+                                     return_argmax=True)
     torch.cuda.synchronize()
     assert dzf.data_ptr() == zv.data_ptr()
     assert torch.equal(rf.loss, ref_r.loss)

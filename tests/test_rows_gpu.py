@@ -357,3 +357,54 @@ def test_repeat_calls_bitwise_identical():
     outs = [ce.ce_forward(zt, yt, 0.1, return_argmax=True) for _ in range(10)]
     for o in outs[1:]:
         assert torch.equal(o.loss, outs[0].loss) and torch.equal(o.lse, outs[0].lse)
+
+
+# ---------------------------------------------------------------------------
+# tiny rows (one or two 16-byte vectors per row): one lane per row
+@pytest.mark.parametrize("V,dt", [(4, "f32"), (8, "f32"), (8, "bf16"), (16, "bf16"),
+                                  (8, "f16"), (16, "f16")])
+def test_tiny_rows(orc, V, dt):
+    N = 1000 + V  # not a multiple of the rows one block takes per step
+    z, z32, y = wl.rows(N, V, dt, seed=300 + V, std=2.0, ignore_frac=0.1)
+    y = y.copy()
+    y[7] = V          # bad target
+    y[14] = 1
+    z32 = z32.copy()
+    z32[11, 1] = np.nan
+    z32[12, :] = -np.inf
+    z32[13, 0] = -np.inf
+    z32[14, :] = 3e36 if dt != "f16" else 6e4   # equal logits at a huge magnitude
+    z32[15, [0, V - 1]] = 5.0                    # argmax tie
+    z, z32 = wl.encode(z32, dt)
+    od = {"f32": None, "bf16": torch.bfloat16, "f16": torch.float16}[dt]
+    for eps, am in ((0.0, True), (0.1, False), (0.2, True)):
+        r, dz = run_fwd_bwd(upload(z, dt), upload(y), eps, out_dtype=od, argmax=am)
+        assert ce.get_error() == 5
+        check_rows(orc, r, dz, z32.astype(np.float64), y, eps, -100, dt, dt)
+        assert abs(r.loss[14].item() - np.log(V)) < 1e-5 * np.log(V) + 1e-6
+
+
+def test_tiny_rows_strided_view_matches_copy(orc):
+    """x[:, :-1] of a (B, L, 8) tensor (rows 32 bytes apart inside a batch,
+    a jump between batches) equals the contiguous copy bit for bit."""
+    x, t = wl.c4a(B=7, L=301, V=8)
+    xt, tt = upload(x), upload(t)
+    r1, d1 = run_fwd_bwd(xt[:, :-1], tt[:, 1:], 0.1)
+    r2, d2 = run_fwd_bwd(xt[:, :-1].contiguous(), tt[:, 1:].contiguous(), 0.1)
+    for a, b in zip(r1, r2):
+        assert torch.equal(a, b)
+    assert torch.equal(d1, d2)
+    z64 = x[:, :-1].reshape(-1, 8).astype(np.float64)
+    check_rows(orc, r1, d1, z64, t[:, 1:].reshape(-1), 0.1, -100, "f32", "f32")
+
+
+def test_tiny_rows_forward_matches_fused():
+    z, _, y = wl.rows(5000, 8, "f32", seed=2, ignore_frac=0.1)
+    zt, yt = upload(z), upload(y)
+    g = torch.full((1,), 0.25, device="cuda")
+    for eps, am in ((0.0, False), (0.1, True)):
+        rs = ce.ce_forward(zt, yt, eps, return_argmax=am)
+        rf, _ = ce.ce_forward_backward(zt, yt, g, eps, return_argmax=am)
+        torch.cuda.synchronize()
+        for a, b in zip(rs, rf):
+            assert (a is None and b is None) or torch.equal(a, b)
