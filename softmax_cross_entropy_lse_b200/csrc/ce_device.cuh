@@ -37,6 +37,14 @@ __device__ __forceinline__ int64_t row_offset(const Layout& L, int64_t r, int64_
     return o * L.s_outer + (r - o * L.inner) * L.s_inner;
 }
 
+// max of three floats in one instruction; like fmaxf, a NaN operand is
+// dropped unless all are NaN.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // Hardware base-2 exponential (MUFU); exp(x) = ex2(x * log2 e).
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -265,14 +273,33 @@ __device__ __forceinline__ void fold(OnlineState& st, const float* v, int col0, 
 template <int U, int VEC, bool MASKED>
 __device__ __forceinline__ void fold_vecs(OnlineState& st, const float (&v)[U][VEC],
                                           const bool (&ok)[U]) {
-    float cm = -INFINITY;
+    // max as a shallow tree: one partial per vector, then across vectors
+    float pm[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
+        pm[u] = -INFINITY;
         if (MASKED && !ok[u]) continue;
+        if constexpr (VEC == 8) {
+            pm[u] = fmaxf(fmax3(v[u][0], v[u][1], v[u][2]),
+                          fmax3(v[u][3], v[u][4], fmax3(v[u][5], v[u][6], v[u][7])));
+        } else if constexpr (VEC == 4) {
+            pm[u] = fmax3(v[u][0], v[u][1], fmaxf(v[u][2], v[u][3]));
+        } else {
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) cm = fmaxf(cm, v[u][e]);
+            for (int e = 0; e < VEC; ++e) pm[u] = fmaxf(pm[u], v[u][e]);
+        }
     }
-    rescale_to(st, fmaxf(st.m, cm));
+#pragma unroll
+    for (int w = U; w > 1; w = (w + 2) / 3) {
+#pragma unroll
+        for (int i = 0; i < (w + 2) / 3; ++i) {
+            const float a = pm[3 * i];
+            const float b = 3 * i + 1 < w ? pm[3 * i + 1] : -INFINITY;
+            const float c = 3 * i + 2 < w ? pm[3 * i + 2] : -INFINITY;
+            pm[i] = fmax3(a, b, c);
+        }
+    }
+    rescale_to(st, fmaxf(st.m, pm[0]));
     const float ms = (st.m == -INFINITY) ? 0.f : st.m;
     int n = 0;
     if constexpr (VEC % 2 == 0) {

@@ -23,9 +23,9 @@ namespace ceb {
 
 // ---------------------------------------------------------------------------
 // Packed rows: G lanes per row, U vectors of VEC elements per lane per step,
-// 32/G rows per warp. The lane whose slice holds column y keeps z_y from its
-// registers (no second, dependent load of the row), and the group adds the
-// one nonzero contribution during the reduction.
+// 32/G rows per warp. The group's first lane, which finalises the row, loads
+// z_y itself as soon as the target is known; the load overlaps the fold, and
+// the other lanes spend nothing on it.
 template <typename T, int VEC, int G, int U, bool ARGMAX, int MINB>
 __global__ void __launch_bounds__(256, MINB) k_fwd_packed(FwdArgs a) {
     const T* __restrict__ z = reinterpret_cast<const T*>(a.z);
@@ -48,9 +48,8 @@ __global__ void __launch_bounds__(256, MINB) k_fwd_packed(FwdArgs a) {
             row = z + row_offset(a.lz, r, a.N);
             y = load_target(a.y, a.tdt, row_offset(a.ly, r, a.N));
         }
-        // column of the target logit, or -1 when there is none to capture
-        const int yc = (y >= 0 && y < a.V && y != a.ignore) ? (int)y : -1;
         float zy = 0.f;
+        if (active && gl == 0 && y >= 0 && y < a.V && y != a.ignore) zy = to_f32(row[y * a.lz.s_col]);
         for (int64_t vb = 0; vb < nvec; vb += (int64_t)G * U) {
             float v[U][VEC];
             bool ok[U];
@@ -71,15 +70,6 @@ __global__ void __launch_bounds__(256, MINB) k_fwd_packed(FwdArgs a) {
                     fold_vecs<U, VEC, true>(st, v, ok);
                     if constexpr (ARGMAX) argmax_vecs<U, VEC, true>(st, v, ok, c0);
                 }
-#pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    const unsigned dy = (unsigned)(yc - c0[u]);
-                    if (ok[u] && dy < (unsigned)VEC) {
-#pragma unroll
-                        for (int e = 0; e < VEC; ++e)
-                            if ((unsigned)e == dy) zy = v[u][e];
-                    }
-                }
             }
         }
         // ragged tail: the last V % VEC columns, one per lane
@@ -89,12 +79,9 @@ __global__ void __launch_bounds__(256, MINB) k_fwd_packed(FwdArgs a) {
                 const int col = (int)(nvec * VEC + q);
                 load_vec<T, 1>(row, col, 1, &x);
                 fold<1, ARGMAX>(st, &x, col, 0);
-                if (col == yc) zy = x;
             }
         }
         group_reduce<G, ARGMAX>(st);
-#pragma unroll
-        for (int off = G / 2; off >= 1; off >>= 1) zy += __shfl_xor_sync(0xffffffffu, zy, off);
         if (active && gl == 0) finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);
     }
 }
@@ -106,12 +93,6 @@ __global__ void __launch_bounds__(256, MINB) k_fwd_packed(FwdArgs a) {
 // is folded in one piece: its max first (three-operand max instructions),
 // then the sum of exponentials, with no running state to rescale. z_y is
 // picked from the registers by a select tree on the bits of the target.
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
 template <int n>
 __device__ __forceinline__ float select_tree(const float (&x)[n], int idx) {
     static_assert((n & (n - 1)) == 0, "power of two");
@@ -556,17 +537,20 @@ __global__ void __launch_bounds__(256) k_fwd_merge(FwdArgs a) {
 template <typename T, int VEC, bool ARGMAX>
 static cudaError_t launch_packed(const FwdArgs& a, int G, int U, int grid, cudaStream_t s) {
     // 32 values per lane per step (8 loads of 4-byte, 4 of 2-byte types);
-    // register budgets for three (4-byte) or two (2-byte) blocks per SM
+    // register budgets for four (4-byte) or two (2-byte) blocks per SM: the
+    // 4-byte rows are latency-bound and gain more from resident warps than
+    // they lose to a few spilled registers (argmax needs three blocks' room)
     constexpr int kU = sizeof(T) == 4 ? 8 : 4;
-    constexpr int kMinB = sizeof(T) == 4 ? 3 : 2;
+    constexpr int kMinB = sizeof(T) == 4 ? (ARGMAX ? 3 : 4) : 2;
+    constexpr int kMinBTiny = sizeof(T) == 4 ? 5 : 4;
 #define CEB_PACKED(GG, UU, MB)                                                    \
     if (G == GG && U == UU) {                                                     \
         k_fwd_packed<T, VEC, GG, UU, ARGMAX, MB><<<grid, 256, 0, s>>>(a);         \
         return cudaGetLastError();                                                \
     }
-    CEB_PACKED(1, 2, 5)  // tiny rows: latency-bound, so as many warps as fit
-    CEB_PACKED(1, kU, kMinB)
-    CEB_PACKED(2, kU, kMinB)
+    CEB_PACKED(1, 2, kMinBTiny)  // tiny rows: latency-bound, so as many warps as fit
+    CEB_PACKED(1, kU, (sizeof(T) == 4 ? 3 : 2))  // fewer rows per warp: more registers
+    CEB_PACKED(2, kU, (sizeof(T) == 4 ? 3 : 2))
     CEB_PACKED(4, kU, kMinB)
     CEB_PACKED(8, kU, kMinB)
     CEB_PACKED(16, kU, kMinB)
