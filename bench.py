@@ -214,60 +214,93 @@ def bench_rows(args, rk):
     bufs = [(z_d, y_d, dz)] + [(z_d.clone(), y_d.clone(), torch.empty_like(dz))
                                for _ in range(nbuf - 1)]
 
-    def step(i, ev=None):
+    def fwd(i):
+        zb, yb, _ = bufs[i % nbuf]
+        zvb, yvb = views(zb, yb)
+        return ce.ce_forward(zvb, yvb, eps, -100, workspace=ws)
+
+    def bwd(i, r):
         zb, yb, db = bufs[i % nbuf]
         zvb, yvb = views(zb, yb)
-        dvb = views(db, yb)[0]
-        if ev is not None:
-            ev[0].record(stream)
-        r = ce.ce_forward(zvb, yvb, eps, -100, workspace=ws)
-        if ev is not None:
-            ev[1].record(stream)
-        ce.ce_backward(g, zvb, yvb, r.lse, r.lse_lo, eps, -100, dlogits=dvb)
-        if ev is not None:
-            ev[2].record(stream)
-        return r
+        ce.ce_backward(g, zvb, yvb, r.lse, r.lse_lo, eps, -100, dlogits=views(db, yb)[0])
+
+    def fused(i):
+        zb, yb, db = bufs[i % nbuf]
+        zvb, yvb = views(zb, yb)
+        ce.ce_forward_backward(zvb, yvb, g, eps, -100, dlogits=views(db, yb)[0], workspace=ws)
 
     fwd_bytes = N * V * esz + 12 * N
     bwd_bytes = 2 * N * V * esz + 12 * N
     step_bytes = fwd_bytes + bwd_bytes
     launches_per_step = (2 if ws_bytes > 0 else 1) + 1
 
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index) as clk:
+    # A batch that fits in L2 takes microseconds on the device, less than the
+    # host needs to issue its calls: its timed loops are captured once as CUDA
+    # graphs and replayed, so the device time is what is measured.
+    use_graph = nbuf > 1
+    fixed = [fwd(i) for i in range(nbuf)]  # saved lse per buffer (backward-only loops)
+
+    def run_loop(kind, steps, ev=None):
+        for i in range(steps):
+            if ev is not None:
+                ev[i][0].record(stream)
+            if kind == "fused":
+                fused(i)
+                continue
+            r = fwd(i) if kind in ("step", "fwd") else fixed[i % nbuf]
+            if ev is not None:
+                ev[i][1].record(stream)
+            if kind in ("step", "bwd"):
+                bwd(i, r)
+            if ev is not None:
+                ev[i][2].record(stream)
+
+    def timed(kind, steps):
+        """Device ms for `steps` iterations (max over ranks); per-iteration
+        events in eager mode."""
+        evs = None
+        if use_graph:
+            gr = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream()
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                run_loop(kind, min(steps, nbuf))
+            stream.wait_stream(side)
+            with torch.cuda.graph(gr):
+                run_loop(kind, steps)
+            gr.replay()
+        else:
+            for i in range(args.warmup):
+                run_loop(kind, 1)
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         sharding.barrier(rk)
         torch.cuda.synchronize()
         t0.record(stream)
-        for i in range(args.steps):
-            step(i, evs[i])
+        if use_graph:
+            gr.replay()
+        else:
+            run_loop(kind, steps, evs)
         t1.record(stream)
         torch.cuda.synchronize()
         sharding.barrier(rk)
-    ms = sharding.max_over_ranks(rk, t0.elapsed_time(t1))
-    fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
-    bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+        return sharding.max_over_ranks(rk, t0.elapsed_time(t1)), evs
 
-    # the same step through the fused call (one read of each short row)
-    fused_ms = None
     for i in range(args.warmup):
-        zb, yb, db = bufs[i % nbuf]
-        zvb, yvb = views(zb, yb)
-        ce.ce_forward_backward(zvb, yvb, g, eps, -100, dlogits=views(db, yb)[0], workspace=ws)
+        run_loop("step", 1)
     torch.cuda.synchronize()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sharding.barrier(rk)
-    f0.record(stream)
-    for i in range(args.steps):
-        zb, yb, db = bufs[i % nbuf]
-        zvb, yvb = views(zb, yb)
-        ce.ce_forward_backward(zvb, yvb, g, eps, -100, dlogits=views(db, yb)[0], workspace=ws)
-    f1.record(stream)
-    torch.cuda.synchronize()
-    fused_ms = sharding.max_over_ranks(rk, f0.elapsed_time(f1)) / args.steps
+    with ClockSampler(dev.index) as clk:
+        ms, evs = timed("step", args.steps)
+    if use_graph:
+        fwd_ms = timed("fwd", args.steps)[0] / args.steps
+        bwd_ms = timed("bwd", args.steps)[0] / args.steps
+    else:
+        fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+        bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+
+    # the same step through the fused call (one read of each row that fits on chip)
+    fused_ms = timed("fused", args.steps)[0] / args.steps
 
     # end to end through the public API with host buffers: pinned host inputs
     # copied in, forward + backward, the per-row loss copied out, every step
@@ -316,7 +349,8 @@ def bench_rows(args, rk):
                    "rows": N, "classes": V, "label_smoothing": eps, "ignore_index": -100,
                    "bytes_per_step": step_bytes,
                    "l2": ("inputs larger than L2" if nbuf == 1 else
-                          f"{nbuf} rotating input buffers (total larger than L2)"),
+                          f"{nbuf} rotating input buffers (total larger than L2); "
+                          "timed loops captured as CUDA graphs and replayed"),
                    "parallelism": f"rows sharded over {world} rank(s), no data-path collective"},
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

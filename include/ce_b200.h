@@ -148,8 +148,8 @@ ce_status ce_backward(const float* grad_out, int64_t grad_stride,
  * there). The logits cross HBM once instead of twice wherever a row fits on
  * chip: rows of up to 1024 elements stay in the registers of the lanes that
  * fold them; longer rows with 16-byte aligned, unit-stride rows (logits and
- * dlogits) and up to 8 x 112 KB per row are copied into shared memory, split
- * over a cluster of 1, 2, 4 or 8 CTAs whose partial states meet once in
+ * dlogits) and up to 4 x 112 KB per row are copied into shared memory, split
+ * over a cluster of 1, 2 or 4 CTAs whose partial states meet once in
  * distributed shared memory, and differentiated from there. Those rows need
  * at least (number of SMs / cluster size) rows per call; otherwise, and for
  * longer or unaligned rows, the call runs the forward, then the backward.

@@ -400,7 +400,9 @@ ce_status ce_forward_backward(const void* logits, ce_dtype dt, ce_layout lg, int
     // to give every SM a CTA); else a forward, then the VJP
     SmemRowPlan sp{};
     if (nvec > (int64_t)kU * G && vec_ok) {
-        for (int cl = 1; cl <= 8; cl *= 2) {
+        // clusters of up to 4 CTAs: rows that need 8 (over 448 KB, e.g. 151,936
+        // fp32) measured slower than the forward followed by the VJP
+        for (int cl = 1; cl <= 4; cl *= 2) {
             const int64_t per = (nvec + cl - 1) / cl;
             const int64_t nch = (per + 127) / 128;
             if (nch <= kSmemRowMaxChunks) {
@@ -453,6 +455,15 @@ ce_status ce_forward_backward(const void* logits, ce_dtype dt, ce_layout lg, int
     const int64_t want = (N + rows_per_block - 1) / rows_per_block;
     const int64_t cap = (int64_t)sms * 16;
     p.grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
+    if (vec_ok && V % vec == 0 && nvec <= 2) {
+        // one or two whole vectors per row: a lane per row, every block resident
+        p.tiny = 1;
+        p.U = (int)nvec;
+        const int64_t rows_tiny = 256 * (int64_t)kTinyRows;
+        const int64_t want_t = (N + rows_tiny - 1) / rows_tiny;
+        const int64_t cap_t = (int64_t)sms * ((nvec == 2 && esz == 2) ? 3 : 4);
+        p.grid = (int)(want_t < cap_t ? (want_t > 0 ? want_t : 1) : cap_t);
+    }
     FusedArgs a{};
     a.f.z = logits;
     a.f.N = N;

@@ -408,6 +408,70 @@ __device__ __forceinline__ void fold_raw16(OnlineState& st, const uint4 (&w)[U],
     }
 }
 
+// A whole row of NV 16-byte words (n = NV * VEC values, all valid) folded in
+// one piece: its max first, then the sum of exponentials, with no running
+// state to rescale. The sums go per vector, then across vectors: the order
+// of fold_vecs, so kernels that fold the same row either way get the same
+// bits. The values are returned in x.
+template <typename T, int VEC, int NV, bool ARGMAX, bool WITH_T>
+__device__ __forceinline__ OnlineState fold_whole_row(const uint4 (&w)[NV], float (&x)[NV * VEC]) {
+    constexpr int n = NV * VEC;
+#pragma unroll
+    for (int v = 0; v < NV; ++v) unpack_words<T>(w[v], x + v * VEC);
+    float m = fmaxf(x[0], x[1]);
+#pragma unroll
+    for (int i = 2; i + 1 < n; i += 2) m = fmax3(m, x[i], x[i + 1]);
+    OnlineState st = empty_state();
+    st.m = m;
+    const float ms = m == -INFINITY ? 0.f : m;
+    const float2 nm = make_float2(-ms, -ms), l2 = make_float2(kLog2e, kLog2e);
+    float2 sa = make_float2(0.f, 0.f), ta = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+        float2 su = make_float2(0.f, 0.f), tu = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = v * VEC; i < (v + 1) * VEC; i += 2) {
+            const float2 d = __fadd2_rn(make_float2(x[i], x[i + 1]), nm);
+            const float2 d2 = __fmul2_rn(d, l2);
+            su = __fadd2_rn(su, make_float2(ex2(d2.x), ex2(d2.y)));
+            if constexpr (WITH_T) tu = __fadd2_rn(tu, d);
+        }
+        sa = __fadd2_rn(sa, su);
+        if constexpr (WITH_T) ta = __fadd2_rn(ta, tu);
+    }
+    st.s = sa.x + sa.y;
+    st.t = ta.x + ta.y;
+    st.k = n;
+    if constexpr (ARGMAX) {
+#pragma unroll
+        for (int i = 0; i < n; ++i) {
+            const float xi = x[i];
+            if ((st.ai < 0) | (xi > st.av) | ((xi != xi) & (st.av == st.av))) {
+                st.av = xi;
+                st.ai = i;
+            }
+        }
+    }
+    return st;
+}
+
+// x[idx] for a power-of-two n by a tree of selects on the bits of idx (no
+// indexed register access).
+template <int n>
+__device__ __forceinline__ float select_tree(const float (&x)[n], int idx) {
+    static_assert((n & (n - 1)) == 0, "power of two");
+    float v[n];
+#pragma unroll
+    for (int i = 0; i < n; ++i) v[i] = x[i];
+#pragma unroll
+    for (int w = n / 2, b = 1; w >= 1; w >>= 1, b <<= 1) {
+        const bool hi = (idx & b) != 0;
+#pragma unroll
+        for (int i = 0; i < w; ++i) v[i] = hi ? v[2 * i + 1] : v[2 * i];
+    }
+    return v[0];
+}
+
 // Argmax over U vectors whose first columns are col0[u], in increasing
 // column order per thread (a strict comparison keeps the first of equals).
 template <int U, int VEC, bool MASKED>

@@ -93,7 +93,8 @@ struct FusedArgs {
 
 struct FusedPlan {
     int vec;
-    int G, U;
+    int G, U;   // tiny: U vectors per row
+    int tiny;   // one lane per row (one or two whole vectors per row)
     int grid;
 };
 

@@ -129,6 +129,87 @@ __global__ void __launch_bounds__(256, MINB) k_fwdbwd_rows(FusedArgs fa) {
     }
 }
 
+// Tiny rows (one or two 16-byte vectors, no ragged tail): one lane per row
+// and R rows per lane per step, every load of the step issued before any is
+// used. The row is folded in one piece exactly as the tiny-row forward folds
+// it (same bits for loss, lse and argmax), and the gradient comes from the
+// same registers.
+template <typename TI, typename TO, int NV, int R, bool ARGMAX, bool WITH_T, int MINB>
+__global__ void __launch_bounds__(256, MINB) k_fwdbwd_tiny(FusedArgs fa) {
+    constexpr int VEC = ElemTraits<TI>::kVec;
+    constexpr int n = NV * VEC;
+    const FwdArgs& a = fa.f;
+    const TI* z = reinterpret_cast<const TI*>(a.z);
+    TO* dz = reinterpret_cast<TO*>(fa.dz);
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const RowOut out{a.loss, a.lse, a.lse_lo, a.argmax, a.err};
+    const float inv_v = 1.f / (float)a.V;
+    const float nan = __int_as_float(0x7fc00000);
+
+    for (int64_t base = warp * 32 * R; base < a.N; base += nwarps * 32 * R) {
+        uint4 w[R][NV];
+        int64_t y[R];
+        float g[R];
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            const int64_t r = base + 32 * k + lane;
+            y[k] = a.ignore;
+            g[k] = 0.f;
+            if (r < a.N) {
+                const TI* row = z + row_offset(a.lz, r, a.N);
+                y[k] = load_target(a.y, a.tdt, row_offset(a.ly, r, a.N));
+                g[k] = fa.g[r * fa.g_stride];
+#pragma unroll
+                for (int v = 0; v < NV; ++v) w[k][v] = __ldcs(reinterpret_cast<const uint4*>(row) + v);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            const int64_t r = base + 32 * k + lane;
+            if (r >= a.N) continue;
+            float x[n];
+            const OnlineState st = fold_whole_row<TI, VEC, NV, ARGMAX, WITH_T>(w[k], x);
+            const int64_t yk = y[k];
+            finalize_row(st, select_tree<n>(x, (int)(yk & (n - 1))), yk, a.ignore, a.V, a.eps, out, r,
+                         ARGMAX);
+            float L, hi, lo;
+            lse_pair(st, L, hi, lo);
+            const bool zero = yk == a.ignore;
+            const bool bad = !zero && (yk < 0 || yk >= a.V);
+            const float gk = g[k];
+            const float c_lo = lo * kLog2e, c_eps = gk * a.eps * inv_v, c_tgt = gk * (1.f - a.eps);
+            float o[n];
+#pragma unroll
+            for (int i = 0; i < n; ++i) {
+                const float p = ex2(fmaf(x[i] - hi, kLog2e, -c_lo));
+                o[i] = (zero || bad) ? (bad ? nan : 0.f) : fmaf(gk, p, -c_eps);
+            }
+            if (!zero && !bad) {
+#pragma unroll
+                for (int i = 0; i < n; ++i)
+                    if (i == yk) o[i] -= c_tgt;
+            }
+            TO* drow = dz + row_offset(fa.ld, r, a.N);
+#pragma unroll
+            for (int v = 0; v < NV; ++v) store_vec<TO, VEC>(drow, v * VEC, 1, o + v * VEC);
+        }
+    }
+}
+
+template <typename TI, typename TO, bool ARGMAX, bool WITH_T>
+static cudaError_t launch_fused_tiny(const FusedPlan& p, const FusedArgs& a, cudaStream_t s) {
+    // register budgets: 64 per thread, 80 for two 16-bit vectors per row
+    if (p.U == 1)
+        k_fwdbwd_tiny<TI, TO, 1, kTinyRows, ARGMAX, WITH_T, 4><<<p.grid, 256, 0, s>>>(a);
+    else if constexpr (sizeof(TI) == 4)
+        k_fwdbwd_tiny<TI, TO, 2, kTinyRows, ARGMAX, WITH_T, 4><<<p.grid, 256, 0, s>>>(a);
+    else
+        k_fwdbwd_tiny<TI, TO, 2, kTinyRows, ARGMAX, WITH_T, 3><<<p.grid, 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
 template <typename TI, typename TO, int VEC, bool ARGMAX>
 static cudaError_t launch_fused_v(const FusedPlan& p, const FusedArgs& a, cudaStream_t s) {
     constexpr int kU = VEC == 1 ? 8 : 32 / VEC;
@@ -152,6 +233,12 @@ static cudaError_t launch_fused_v(const FusedPlan& p, const FusedArgs& a, cudaSt
 template <typename TI, typename TO>
 static cudaError_t launch_fused_t(const FusedPlan& p, const FusedArgs& a, cudaStream_t s) {
     const bool am = a.f.argmax != nullptr;
+    if (p.tiny) {
+        const bool t = a.f.eps != 0.f;
+        if (am)
+            return t ? launch_fused_tiny<TI, TO, true, true>(p, a, s) : launch_fused_tiny<TI, TO, true, false>(p, a, s);
+        return t ? launch_fused_tiny<TI, TO, false, true>(p, a, s) : launch_fused_tiny<TI, TO, false, false>(p, a, s);
+    }
     if (p.vec == 1)
         return am ? launch_fused_v<TI, TO, 1, true>(p, a, s) : launch_fused_v<TI, TO, 1, false>(p, a, s);
     constexpr int V8 = ElemTraits<TI>::kVec;

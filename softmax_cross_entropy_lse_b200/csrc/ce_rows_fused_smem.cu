@@ -1,5 +1,5 @@
 // Fused forward + VJP for rows held in shared memory (rows too long for one
-// warp's registers, up to 8 x 112 KB).
+// warp's registers, up to 4 x 112 KB).
 //
 // When g is known before the forward runs, the gradient
 //     dz_j = g (exp(z_j - lse) - (1 - eps)[j = y] - eps/V)
@@ -12,7 +12,7 @@
 // the saved lse, section 1 of the same page).
 //
 // A row longer than one CTA's share of shared memory is split across a
-// thread-block cluster of CL CTAs (CL = 1, 2, 4, 8); CTA k holds vectors
+// thread-block cluster of CL CTAs (CL = 1, 2, 4); CTA k holds vectors
 // [k S, (k+1) S) of the row. Each CTA reduces its slice, the CL partial
 // states are exchanged once through distributed shared memory, and every CTA
 // merges them in rank order, so all of them derive the same lse bits.
@@ -346,7 +346,6 @@ static cudaError_t launch_smem_cl(const SmemRowPlan& sp, const FusedArgs& a, cud
         case 1: return launch_smem_k<TI, TO, 1, ARGMAX, WITH_T>(sp, a, s);
         case 2: return launch_smem_k<TI, TO, 2, ARGMAX, WITH_T>(sp, a, s);
         case 4: return launch_smem_k<TI, TO, 4, ARGMAX, WITH_T>(sp, a, s);
-        case 8: return launch_smem_k<TI, TO, 8, ARGMAX, WITH_T>(sp, a, s);
     }
     return cudaErrorInvalidValue;
 }

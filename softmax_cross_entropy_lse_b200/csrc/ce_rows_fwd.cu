@@ -93,21 +93,6 @@ __global__ void __launch_bounds__(256, MINB) k_fwd_packed(FwdArgs a) {
 // is folded in one piece: its max first (three-operand max instructions),
 // then the sum of exponentials, with no running state to rescale. z_y is
 // picked from the registers by a select tree on the bits of the target.
-template <int n>
-__device__ __forceinline__ float select_tree(const float (&x)[n], int idx) {
-    static_assert((n & (n - 1)) == 0, "power of two");
-    float v[n];
-#pragma unroll
-    for (int i = 0; i < n; ++i) v[i] = x[i];
-#pragma unroll
-    for (int w = n / 2, b = 1; w >= 1; w >>= 1, b <<= 1) {
-        const bool hi = (idx & b) != 0;
-#pragma unroll
-        for (int i = 0; i < w; ++i) v[i] = hi ? v[2 * i + 1] : v[2 * i];
-    }
-    return v[0];
-}
-
 template <typename T, int VEC, int NV, int R, bool ARGMAX, bool WITH_T, int MINB>
 __global__ void __launch_bounds__(256, MINB) k_fwd_tiny(FwdArgs a) {
     constexpr int n = NV * VEC;
@@ -136,44 +121,7 @@ __global__ void __launch_bounds__(256, MINB) k_fwd_tiny(FwdArgs a) {
             const int64_t r = base + 32 * k + lane;
             if (r >= a.N) continue;
             float x[n];
-#pragma unroll
-            for (int v = 0; v < NV; ++v) unpack_words<T>(w[k][v], x + v * VEC);
-            float m = fmaxf(x[0], x[1]);
-#pragma unroll
-            for (int i = 2; i + 1 < n; i += 2) m = fmax3(m, x[i], x[i + 1]);
-            OnlineState st = empty_state();
-            st.m = m;
-            const float ms = m == -INFINITY ? 0.f : m;
-            const float2 nm = make_float2(-ms, -ms), l2 = make_float2(kLog2e, kLog2e);
-            // per-vector partial pairs, then across vectors: the order of
-            // fold_vecs, so the fused forward + VJP gets the same bits
-            float2 sa = make_float2(0.f, 0.f), ta = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int v = 0; v < NV; ++v) {
-                float2 su = make_float2(0.f, 0.f), tu = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int i = v * VEC; i < (v + 1) * VEC; i += 2) {
-                    const float2 d = __fadd2_rn(make_float2(x[i], x[i + 1]), nm);
-                    const float2 d2 = __fmul2_rn(d, l2);
-                    su = __fadd2_rn(su, make_float2(ex2(d2.x), ex2(d2.y)));
-                    if constexpr (WITH_T) tu = __fadd2_rn(tu, d);
-                }
-                sa = __fadd2_rn(sa, su);
-                if constexpr (WITH_T) ta = __fadd2_rn(ta, tu);
-            }
-            st.s = sa.x + sa.y;
-            st.t = ta.x + ta.y;
-            st.k = n;
-            if constexpr (ARGMAX) {
-#pragma unroll
-                for (int i = 0; i < n; ++i) {
-                    const float xi = x[i];
-                    if ((st.ai < 0) | (xi > st.av) | ((xi != xi) & (st.av == st.av))) {
-                        st.av = xi;
-                        st.ai = i;
-                    }
-                }
-            }
+            const OnlineState st = fold_whole_row<T, VEC, NV, ARGMAX, WITH_T>(w[k], x);
             const int64_t yk = y[k];
             const float zy = select_tree<n>(x, (int)(yk & (n - 1)));
             finalize_row(st, zy, yk, a.ignore, a.V, a.eps, out, r, ARGMAX);

@@ -151,7 +151,8 @@ def _padded(N, V, pad, dtype, seed, std=2.0, ignore_frac=0.1):
     (100000, 200, "bf16"),     # cluster of 2
     (151936, 160, "bf16"),     # cluster of 4, the 2048 x 151,936 row shape
     (20000, 300, "f32"),       # one CTA, fp32
-    (151936, 40, "f32"),       # cluster of 8, fp32
+    (100000, 80, "f32"),       # cluster of 4, fp32
+    (151936, 40, "f32"),       # 608 KB rows: the forward, then the VJP
 ])
 def test_smem_rows_vs_oracle(orc, V, N, dt):
     z, z32, y = wl.rows(N, V, dt, seed=V % 997 + N, std=2.0, ignore_frac=0.1)
@@ -194,7 +195,7 @@ def test_smem_rows_ragged_tail_views(orc, out):
 
 def test_smem_rows_strided_3d_view_cluster(orc):
     """The (B, L, V) view x[:, :-1] at V = 151,936 fp32 (rows of 607,744 bytes,
-    a cluster of 8 CTAs per row), targets t[:, 1:]."""
+    beyond four CTAs' shared memory: the forward, then the VJP), targets t[:, 1:]."""
     x, t = wl.c4a(B=3, L=21, V=151936)
     xt, tt = upload(x), upload(t)
     zv, yv = xt[:, :-1], tt[:, 1:]
@@ -241,3 +242,54 @@ def test_smem_rows_bad_targets_and_nonfinite(orc):
     torch.cuda.synchronize()
     assert ce.get_error() == 5
     check_oracle(orc, rf, dzf, z32.astype(np.float64), y, 1.0, 0.0, -100, "f32", "f32")
+
+
+# -- tiny rows (one or two 16-byte vectors): one lane per row --------------------------------
+@pytest.mark.parametrize("V,dt,out", [(4, "f32", "f32"), (8, "f32", "f32"), (8, "bf16", "bf16"),
+                                      (16, "bf16", "f32"), (8, "f16", "f16"), (16, "f16", "f16")])
+def test_tiny_rows_fused(orc, V, dt, out):
+    N = 3000 + V
+    z, z32, y = wl.rows(N, V, dt, seed=40 + V, std=2.0, ignore_frac=0.1)
+    y = y.copy()
+    y[3] = -5                     # bad target
+    y[9] = 0
+    z32 = z32.copy()
+    z32[4, 1] = np.nan
+    z32[5, :] = -np.inf
+    z32[6, 0] = -np.inf
+    z32[9, :] = 1e4
+    z, z32 = wl.encode(z32, dt)
+    gv = np.random.default_rng(V).standard_normal(N).astype(np.float32)
+    zt, yt, gt = upload(z, dt), upload(y), upload(gv)
+    od = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[out]
+    for eps, am in ((0.0, True), (0.1, False)):
+        rf, dzf = ce.ce_forward_backward(zt, yt, gt, eps, return_argmax=am, out_dtype=od)
+        rs = ce.ce_forward(zt, yt, eps, return_argmax=am)
+        torch.cuda.synchronize()
+        assert ce.get_error() == 5
+        for a, b in zip(rf, rs):  # bit for bit, NaN rows included
+            assert (a is None and b is None) or torch.equal(a.view(torch.int32), b.view(torch.int32))
+        loss, lse, amx = orc.ce_forward(z32.astype(np.float64), y, eps)
+        rt, at = loss_tol(dt)
+        assert_close(f32(rf.loss), loss, rt, at, "loss")
+        assert_close(f32(rf.lse), lse, rt, at, "lse")
+        if am:
+            np.testing.assert_array_equal(rf.argmax.cpu().numpy(), amx)
+        ref = orc.ce_backward(z32.astype(np.float64), y, gv.astype(np.float64), eps)
+        assert_grad_close(f32(dzf), ref, dt, out)
+
+
+def test_tiny_rows_fused_in_place_view(orc):
+    """In place on the (B, L, 8) view x[:, :-1]."""
+    x, t = wl.c4a(B=5, L=97, V=8)
+    xt, tt = upload(x), upload(t)
+    zv, yv = xt[:, :-1], tt[:, 1:]
+    rf, dzf = ce.ce_forward_backward(zv, yv, torch.ones(1, device="cuda"), 0.1, dlogits=zv)
+    torch.cuda.synchronize()
+    assert dzf.data_ptr() == zv.data_ptr()
+    z64 = x[:, :-1].reshape(-1, 8).astype(np.float64)
+    y = t[:, 1:].reshape(-1)
+    loss, _, _ = orc.ce_forward(z64, y, 0.1)
+    assert_close(f32(rf.loss), loss, 1e-5, 1e-6, "loss")
+    ref = orc.ce_backward(z64, y, 1.0, 0.1)
+    assert_grad_close(f32(zv).reshape(-1, 8), ref, "f32", "f32")
