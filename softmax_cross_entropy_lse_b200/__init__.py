@@ -185,9 +185,32 @@ def ce_workspace_size(N: int, V: int, dtype, num_sms: int = 0) -> int:
     return int(lib().ce_workspace_size(N, V, code, num_sms))
 
 
+def _row_outputs(N: int, dev, return_argmax: bool, out):
+    """Per-row output tensors: fresh ones, or the caller's `out` (a
+    ForwardResult of contiguous float32 loss, lse, lse_lo and int32 argmax on
+    the logits' device, N entries each), written in place."""
+    torch = _torch()
+    if out is None:
+        return (torch.empty(N, dtype=torch.float32, device=dev),
+                torch.empty(N, dtype=torch.float32, device=dev),
+                torch.empty(N, dtype=torch.float32, device=dev),
+                torch.empty(N, dtype=torch.int32, device=dev) if return_argmax else None)
+    loss, lse, lse_lo, am = out
+    want = [(loss, torch.float32), (lse, torch.float32), (lse_lo, torch.float32)]
+    if return_argmax:
+        if am is None:
+            raise ValueError("return_argmax needs an argmax tensor in `out`")
+        want.append((am, torch.int32))
+    for t, dt in want:
+        if t.dtype != dt or t.numel() != N or not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"`out` tensors must be contiguous {dt} with {N} entries on {dev}")
+    return loss, lse, lse_lo, (am if return_argmax else None)
+
+
 def ce_forward(logits, targets, label_smoothing: float = 0.0, ignore_index: int = -100, *,
-               return_argmax: bool = False, workspace=None, stream=None) -> ForwardResult:
-    """Per-row loss, lse (and its low-order float lse_lo, and optional argmax)."""
+               return_argmax: bool = False, workspace=None, stream=None, out=None) -> ForwardResult:
+    """Per-row loss, lse (and its low-order float lse_lo, and optional argmax).
+    `out` (a ForwardResult) receives them in place instead of new tensors."""
     torch = _torch()
     _require_cuda(logits, targets)
     N, lg = row_layout(logits, True)
@@ -196,10 +219,7 @@ def ce_forward(logits, targets, label_smoothing: float = 0.0, ignore_index: int 
         raise ValueError(f"targets hold {Nt} rows, logits {N}")
     V = logits.shape[-1]
     dev = logits.device
-    loss = torch.empty(N, dtype=torch.float32, device=dev)
-    lse = torch.empty(N, dtype=torch.float32, device=dev)
-    lse_lo = torch.empty(N, dtype=torch.float32, device=dev)
-    am = torch.empty(N, dtype=torch.int32, device=dev) if return_argmax else None
+    loss, lse, lse_lo, am = _row_outputs(N, dev, return_argmax, out)
     dt = _dtype_code(logits)
     with torch.cuda.device(dev):
         need = int(lib().ce_workspace_size(N, V, dt, 0))
@@ -256,9 +276,10 @@ def ce_backward(grad_out, logits, targets, lse, lse_lo=None, label_smoothing: fl
 
 def ce_forward_backward(logits, targets, grad_out, label_smoothing: float = 0.0,
                         ignore_index: int = -100, *, return_argmax: bool = False, dlogits=None,
-                        out_dtype=None, workspace=None, stream=None):
+                        out_dtype=None, workspace=None, stream=None, out=None):
     """Forward and VJP in one call (g known up front). Returns (ForwardResult,
-    dlogits); short rows are read from HBM once."""
+    dlogits); rows that fit on chip are read from HBM once. `out` as for
+    ce_forward."""
     torch = _torch()
     _require_cuda(logits, targets, grad_out, dlogits)
     N, lg = row_layout(logits, True)
@@ -280,10 +301,7 @@ def ce_forward_backward(logits, targets, grad_out, label_smoothing: float = 0.0,
     Nd, dl = row_layout(dlogits, True)
     if Nd != N or dlogits.shape[-1] != V:
         raise ValueError("dlogits must have the shape of logits")
-    loss = torch.empty(N, dtype=torch.float32, device=dev)
-    lse = torch.empty(N, dtype=torch.float32, device=dev)
-    lse_lo = torch.empty(N, dtype=torch.float32, device=dev)
-    am = torch.empty(N, dtype=torch.int32, device=dev) if return_argmax else None
+    loss, lse, lse_lo, am = _row_outputs(N, dev, return_argmax, out)
     dt = _dtype_code(logits)
     with torch.cuda.device(dev):
         need = int(lib().ce_workspace_size(N, V, dt, 0))

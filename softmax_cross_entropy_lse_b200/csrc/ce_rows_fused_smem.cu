@@ -19,10 +19,10 @@
 //
 // Within a CTA, 8 warps own the 2 KB chunks of the slice round-robin (chunk c
 // belongs to warp c % 8). A warp's lane 0 copies its chunks in with 1-D bulk
-// copies (TMA engine), the warp folds them as they land, and after the
-// gradient pass over a chunk it refills that chunk with the next row's bytes
-// at once: no CTA-wide barrier guards the buffers, and the next row streams
-// in while this one is being differentiated. The warp and CTA states of row
+// copies (TMA engine), the warp folds them as they land, and once its
+// gradient pass over them is done it refills them with the next row's bytes:
+// no CTA-wide barrier guards the buffers, and the next row streams in while
+// the other warps are still differentiating this one. The warp and CTA states of row
 // i use exchange slots of parity i & 1, so no slot is rewritten before every
 // reader has passed the next barrier (the race of Suryavanshi, "One barrier
 // short", cannot occur). Every wait is bounded; on expiry the kernel raises
@@ -251,14 +251,17 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
         const float c_lo = lo * kLog2e, c_eps = g * a.eps * inv_v, c_tgt = g * (1.f - a.eps);
         const int cst_mode = bad ? 2 : (ign ? 1 : 0);
         const int64_t rn = r + ncl;
-        for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps) {
+        for (int c = wid; c < nch; c += kSmWarps) {
             if (!dead)
                 grad_chunk<TI, TO>(chunk_buf(c), chunk_vecs(c), lane, v0 + (int64_t)c * kSmChunkVecs,
                                    drow, hi, c_lo, g, c_eps, c_tgt, yc, cst_mode);
-            // the chunk is read: refill it with the next row's bytes
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (rn < a.N && !dead) {
+        }
+        // this warp's chunks are read: refill them with the next row's bytes
+        // (one proxy fence for all of them)
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (rn < a.N && !dead) {
+            for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps) {
                 if (lane == 0) issue(rn, c);
                 pend |= 1u << i;
             }

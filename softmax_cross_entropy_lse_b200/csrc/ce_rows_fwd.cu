@@ -228,7 +228,15 @@ __global__ void __launch_bounds__(kCtaThreads, kCtaMinBlocks) k_fwd_cta(FwdArgs 
 // boundaries), and the lanes fold each chunk straight from shared memory. The
 // bytes in flight per SM are set by the rings (up to 192 KB), not by the
 // registers of the folding threads. Chunk c of a unit belongs to warp
-// c % kRingWarps; the warps of a unit meet once, in one exchange of states.
+// c % kRingWarps; the warps of a unit meet once, in one exchange of states:
+// each warp writes its state to a slot and arrives on a named barrier without
+// waiting, and only the unit's finaliser (a role that rotates over the warps)
+// waits for all of them, merges and writes the row. Slots alternate between
+// two sets; the finaliser releases its set through a second named barrier,
+// which the other warps pass before they write that set again two units
+// later (so no slot is rewritten before it is read: the race of "One barrier
+// short" cannot occur), and the warps of a CTA stay within two units of each
+// other, streaming neighbouring parts of the same rows.
 constexpr int kRingWarps = 8;
 constexpr int kRingStages = 4;
 constexpr int kRingVecs = 128;  // 2 KB per stage
@@ -332,14 +340,18 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
     uint32_t consumed = 0, waited = 0;
     bool dead = false;
     int parity = 0;
-    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, parity ^= 1) {
+    uint32_t it = 0;  // units of this CTA so far
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, parity ^= 1, ++it) {
         const RingUnit ru = ring_unit<T>(a, u, nvec);
         const int64_t r = a.splits == 1 ? u : u / a.splits;
         const int sp = a.splits == 1 ? 0 : (int)(u - r * a.splits);
         const T* row = reinterpret_cast<const T*>(a.z) + row_offset(a.lz, r, a.N);
+        // the unit's finaliser rotates over the warps; it fetches the target
+        // and its logit up front
+        const int fin = (int)(it % kRingWarps);
         int64_t y = 0;
         float zy = 0.f;
-        if (a.splits == 1 && tid == 0) {
+        if (a.splits == 1 && wid == fin && lane == 0) {
             y = load_target(a.y, a.tdt, row_offset(a.ly, r, a.N));
             if (y != a.ignore && y >= 0 && y < a.V) zy = to_f32(row[y]);
         }
@@ -412,11 +424,18 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
             }
         }
         group_reduce<32, ARGMAX, WITH_T>(st);
+        // slot[parity] was last read by the finaliser of unit it - 2; every
+        // other warp waits for its release before overwriting it
+        if (it >= 2 && wid != (int)((it - 2) % kRingWarps)) named_bar_sync(3 + parity, kRingWarps * 32);
         if (lane == 0) slots[parity][wid] = st;
-        __syncthreads();
-        if (wid == 0) {
+        if (wid != fin) {
+            named_bar_arrive(1 + parity, kRingWarps * 32);
+        } else {
+            named_bar_sync(1 + parity, kRingWarps * 32);
             st = slots[parity][lane & (kRingWarps - 1)];
             group_reduce<kRingWarps, ARGMAX, WITH_T>(st);
+            // the slots are read: release them for unit it + 2, if this CTA has one
+            if ((int64_t)u + 2 * (int64_t)gridDim.x < units) named_bar_arrive(3 + parity, kRingWarps * 32);
             if (lane == 0) {
                 if (a.splits == 1) {
                     finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);

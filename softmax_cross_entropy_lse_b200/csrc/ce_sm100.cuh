@@ -138,6 +138,18 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ---- named barriers ----------------------------------------------------------------
+// Barrier `id` (1..15; 0 is __syncthreads) completes when `count` threads
+// (a multiple of 32, whole warps) have arrived. arrive does not wait; it
+// orders the thread's earlier memory accesses before the barrier for the
+// threads that sync on it.
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ---- thread-block clusters and distributed shared memory ---------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;

@@ -172,3 +172,18 @@ def test_row_layout_marshalling():
     assert N == 64 and lg.s_inner == 1 and lg.s_col == 64
     with pytest.raises(ValueError):
         ce.row_layout(torch.empty(4, 5, 6, 7)[:, :-1, :-1], True)
+
+
+def test_out_tensors_validated():
+    """ce_forward(out=...) checks the caller's tensors before any launch."""
+    import torch
+    import softmax_cross_entropy_lse_b200 as ce
+    good = ce.ForwardResult(*(torch.empty(5) for _ in range(3)), None)
+    assert ce._row_outputs(5, torch.device("cpu"), False, good)[0] is good.loss
+    for bad in (ce.ForwardResult(torch.empty(4), torch.empty(5), torch.empty(5), None),
+                ce.ForwardResult(torch.empty(5, dtype=torch.float64), torch.empty(5), torch.empty(5), None),
+                ce.ForwardResult(torch.empty(10)[::2], torch.empty(5), torch.empty(5), None)):
+        with pytest.raises(ValueError):
+            ce._row_outputs(5, torch.device("cpu"), False, bad)
+    with pytest.raises(ValueError):
+        ce._row_outputs(5, torch.device("cpu"), True, good)  # argmax requested, none given

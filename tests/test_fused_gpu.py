@@ -193,7 +193,7 @@ def test_smem_rows_ragged_tail_views(orc, out):
     check_oracle(orc, rf, dzf, z32.astype(np.float64), y, 1.0, 0.2, -100, "bf16", out)
 
 
-def test_smem_rows_strided_3d_view_cluster(orc):
+def test_long_rows_strided_3d_view(orc):
     """The (B, L, V) view x[:, :-1] at V = 151,936 fp32 (rows of 607,744 bytes,
     beyond four CTAs' shared memory: the forward, then the VJP), targets t[:, 1:]."""
     x, t = wl.c4a(B=3, L=21, V=151936)

@@ -408,3 +408,23 @@ def test_tiny_rows_forward_matches_fused():
         torch.cuda.synchronize()
         for a, b in zip(rs, rf):
             assert (a is None and b is None) or torch.equal(a, b)
+
+
+def test_forward_into_caller_outputs():
+    """out=: the per-row results land in the caller's tensors, bit for bit the
+    same as freshly allocated ones, for the forward and the fused call."""
+    z, _, y = wl.rows(700, 3000, "bf16", seed=21, std=2.0, ignore_frac=0.1)
+    zt, yt = upload(z, "bf16"), upload(y)
+    out = ce.ForwardResult(*(torch.full((700,), float("nan"), device="cuda") for _ in range(3)),
+                           torch.full((700,), -1, dtype=torch.int32, device="cuda"))
+    ref = ce.ce_forward(zt, yt, 0.1, return_argmax=True)
+    got = ce.ce_forward(zt, yt, 0.1, return_argmax=True, out=out)
+    torch.cuda.synchronize()
+    for a, b, c in zip(ref, got, out):
+        assert b.data_ptr() == c.data_ptr() and torch.equal(a, b)
+    g = torch.ones(1, device="cuda")
+    ref2, _ = ce.ce_forward_backward(zt, yt, g, 0.1, return_argmax=True)
+    got2, _ = ce.ce_forward_backward(zt, yt, g, 0.1, return_argmax=True, out=out)
+    torch.cuda.synchronize()
+    for a, b, c in zip(ref2, got2, out):
+        assert b.data_ptr() == c.data_ptr() and torch.equal(a, b)
