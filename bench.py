@@ -63,10 +63,18 @@ def load_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def kernel_source_sha() -> str:
+# Source files each pass's kernels are built from (the shared device code,
+# the launch interface, the planner and the pass's own file).
+PASS_SOURCES = {
+    "forward": ["ce_rows_fwd.cu", "ce_device.cuh", "ce_launch.h", "ce_api.cu", "ce_sm100.cuh"],
+    "backward": ["ce_rows_bwd.cu", "ce_device.cuh", "ce_launch.h", "ce_api.cu", "ce_sm100.cuh"],
+}
+
+
+def kernel_source_sha(files) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "softmax_cross_entropy_lse_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode())
             h.update(fh.read())
@@ -75,14 +83,14 @@ def kernel_source_sha() -> str:
 
 def recorded_traffic(workload: str, kernel: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
+    the current sources of that pass's kernels; else None."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
-    if not os.path.exists(p):
+    if not os.path.exists(p) or kernel not in PASS_SOURCES:
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(workload, {}).get(kernel)
-    if not e or e.get("source_sha") != kernel_source_sha():
+    if not e or e.get("source_sha") != kernel_source_sha(PASS_SOURCES[kernel]):
         return None
     return e.get("bytes_per_launch")
 
