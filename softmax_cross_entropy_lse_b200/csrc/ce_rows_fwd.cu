@@ -102,9 +102,19 @@ __global__ void __launch_bounds__(256, MINB) k_fwd_tiny(FwdArgs a) {
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const RowOut out{a.loss, a.lse, a.lse_lo, a.argmax, a.err};
 
+    // rows lie back to back in memory when the layout is a plain matrix
+    const bool dense = a.lz.inner >= a.N && a.lz.s_inner == (int64_t)n;
     for (int64_t base = warp * 32 * R; base < a.N; base += nwarps * 32 * R) {
         uint4 w[R][NV];
         int64_t y[R];
+        if (dense && lane == 0) {
+            // the warp's next step (32 R rows) starts moving into L2 now
+            const int64_t bn = base + nwarps * 32 * R;
+            if (bn < a.N) {
+                const int64_t rows = min((int64_t)32 * R, a.N - bn);
+                sm100::bulk_prefetch_l2(z + bn * n, (uint32_t)(rows * n * sizeof(T)));
+            }
+        }
 #pragma unroll
         for (int k = 0; k < R; ++k) {
             const int64_t r = base + 32 * k + lane;
