@@ -53,6 +53,8 @@ class Oracle:
                                             _f64p, ctypes.c_double, _i64, _f64p]
         L.orc_linear_ce_backward.argtypes = [_f32p, _f32p, _i64, _i64, _i64, _i64p, _f64p,
                                              ctypes.c_double, _i64, _f64p, _f64p, _f64p]
+        L.orc_ce_soft_forward.argtypes = [_f64p, _f64p, _i64, _i64, ctypes.c_double, _f64p, _f64p]
+        L.orc_ce_soft_backward.argtypes = [_f64p, _f64p, _i64, _i64, _f64p, ctypes.c_double, _f64p]
         L.orc_num_threads.restype = ctypes.c_int
 
     # -- helpers -----------------------------------------------------------
@@ -84,6 +86,31 @@ class Oracle:
         self.lib.orc_ce_backward(self._p(z, _f64p), N, V, self._p(y, _i64p),
                                  self._p(g, _f64p), float(eps), int(ignore_index),
                                  self._p(dz, _f64p))
+        return dz
+
+    # -- probability (soft) targets ----------------------------------------
+    def ce_soft_forward(self, z, t, eps: float = 0.0):
+        """loss, lse (float64, N) of each row of z (N, V) against the target
+        distribution t (N, V): loss = sum_j t'_j (lse - z_j)."""
+        z = np.ascontiguousarray(z, dtype=np.float64)
+        t = np.ascontiguousarray(t, dtype=np.float64)
+        N, V = z.shape
+        assert t.shape == (N, V)
+        loss = np.empty(N, np.float64)
+        lse = np.empty(N, np.float64)
+        self.lib.orc_ce_soft_forward(self._p(z, _f64p), self._p(t, _f64p), N, V, float(eps),
+                                     self._p(loss, _f64p), self._p(lse, _f64p))
+        return loss, lse
+
+    def ce_soft_backward(self, z, t, g, eps: float = 0.0):
+        """Gradient of sum_i g_i loss_i with respect to z, float64 (N, V)."""
+        z = np.ascontiguousarray(z, dtype=np.float64)
+        t = np.ascontiguousarray(t, dtype=np.float64)
+        N, V = z.shape
+        g = np.ascontiguousarray(np.broadcast_to(np.asarray(g, np.float64), (N,)))
+        dz = np.empty((N, V), np.float64)
+        self.lib.orc_ce_soft_backward(self._p(z, _f64p), self._p(t, _f64p), N, V,
+                                      self._p(g, _f64p), float(eps), self._p(dz, _f64p))
         return dz
 
     # -- fused-linear cross-entropy ---------------------------------------

@@ -250,6 +250,88 @@ void orc_linear_ce_backward(const float* H, const float* W, int64_t N,
     }
 }
 
+/* ---- Probability (soft) targets --------------------------------------------
+ * The cross-entropy of the softmax of a row z against a target distribution
+ * t over the same V classes (MLX PR #4188, "Shift by the max in
+ * cross_entropy": the loss is lse minus the target-weighted logits, assembled
+ * from shifted values):
+ *     loss = sum_j t'_j (lse - z_j),   t'_j = (1-eps) t_j + eps/V,
+ * which is lse - sum_j t_j z_j when t sums to 1 and eps = 0. Its gradient
+ * with respect to z_k, scaled by g, is
+ *     dz_k = g (p_k T' - t'_k),   p_k = exp(z_k - lse),   T' = sum_j t'_j.
+ * Readings where the pages are silent:
+ *   - t is used as given (not renormalised; negative entries allowed).
+ *   - label smoothing mixes t with the uniform distribution, as for hard
+ *     targets: eps/V on every class.
+ *   - a class whose t'_j is exactly 0 contributes nothing, even where z_j is
+ *     -inf (the 0 log 0 = 0 convention of cross-entropy).
+ *   - NaN anywhere in z, or a row of z that is all -inf: lse as for hard
+ *     targets (NaN, -inf), loss NaN, gradient row NaN.
+ *   - there is no ignore_index. */
+static void soft_row_forward(const double* z, const double* t, int64_t V, double eps,
+                             double* loss, double* lse, double* m_out, double* s_out)
+{
+    double m = -INFINITY;
+    for (int64_t j = 0; j < V; ++j) {
+        if (isnan(z[j])) { m = NAN; break; }
+        if (z[j] > m) m = z[j];
+    }
+    *m_out = m;
+    if (isnan(m) || m == -INFINITY) {
+        *lse = isnan(m) ? NAN : -INFINITY;
+        *loss = NAN;
+        *s_out = isnan(m) ? NAN : 0.0;
+        return;
+    }
+    double s = 0.0;
+    for (int64_t j = 0; j < V; ++j) s += exp(z[j] - m);
+    const double L = log(s);
+    *lse = m + L;
+    *s_out = s;
+    double l = 0.0;
+    for (int64_t j = 0; j < V; ++j) {
+        const double tj = (1.0 - eps) * t[j] + eps / (double)V;
+        if (tj != 0.0) l += tj * (L - (z[j] - m));
+    }
+    *loss = l;
+}
+
+/* Soft-target forward over contiguous (N, V) logits and targets. */
+void orc_ce_soft_forward(const double* z, const double* t, int64_t N, int64_t V, double eps,
+                         double* loss, double* lse)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i) {
+        double m, s;
+        soft_row_forward(z + i * V, t + i * V, V, eps, &loss[i], &lse[i], &m, &s);
+    }
+}
+
+/* Soft-target VJP: dz_k = g_i (p_k T' - t'_k). g: N doubles; dz: N*V. */
+void orc_ce_soft_backward(const double* z, const double* t, int64_t N, int64_t V,
+                          const double* g, double eps, double* dz)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i) {
+        const double* zr = z + i * V;
+        const double* tr = t + i * V;
+        double* d = dz + i * V;
+        double loss, lse, m, s;
+        soft_row_forward(zr, tr, V, eps, &loss, &lse, &m, &s);
+        if (isnan(m) || m == -INFINITY) {
+            for (int64_t j = 0; j < V; ++j) d[j] = NAN;
+            continue;
+        }
+        double T = 0.0;
+        for (int64_t j = 0; j < V; ++j) T += (1.0 - eps) * tr[j] + eps / (double)V;
+        for (int64_t j = 0; j < V; ++j) {
+            const double p = exp(zr[j] - m) / s;
+            const double tj = (1.0 - eps) * tr[j] + eps / (double)V;
+            d[j] = g[i] * (p * T - tj);
+        }
+    }
+}
+
 /* Threads OpenMP will use, for reporting the CPU baseline's core count. */
 int orc_num_threads(void)
 {

@@ -17,6 +17,9 @@ Sources of truth used here:
     and its autograd, as an independent library special case.
   * Central finite differences of the oracle's own forward.
   * numpy float64 matmul for Z = H W^T and for G W, G^T H (library step).
+  * For probability targets: the hard-target oracle at one-hot targets, PyTorch's
+    float64 cross_entropy with probability targets, closed forms, shift
+    invariance and finite differences.
 """
 from __future__ import annotations
 
@@ -312,6 +315,125 @@ def pin_linear_finite_differences(orc):
             np.testing.assert_allclose(dA, fd, rtol=0, atol=5e-7)
 
 
+# ---- probability (soft) targets ---------------------------------------------------
+def _soft_draw(rng, N, V, normalised=True):
+    z = rng.standard_normal((N, V))
+    t = rng.random((N, V))
+    if normalised:
+        t /= t.sum(1, keepdims=True)
+    return z, t
+
+
+def pin_soft_onehot_matches_hard(orc):
+    """A one-hot target distribution is the hard target: same loss, lse and
+    gradient, with and without label smoothing."""
+    rng = np.random.default_rng(31)
+    N, V = 9, 13
+    z = rng.standard_normal((N, V)) * 3
+    y = rng.integers(0, V, size=N)
+    t = np.zeros((N, V))
+    t[np.arange(N), y] = 1.0
+    g = rng.standard_normal(N)
+    for eps in (0.0, 0.3):
+        ls, lses = orc.ce_soft_forward(z, t, eps)
+        lh, lseh, _ = orc.ce_forward(z, y, eps)
+        np.testing.assert_allclose(ls, lh, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(lses, lseh, rtol=1e-15)
+        np.testing.assert_allclose(orc.ce_soft_backward(z, t, g, eps), orc.ce_backward(z, y, g, eps),
+                                   rtol=1e-12, atol=1e-15)
+
+
+def pin_soft_torch_float64(orc):
+    """PyTorch's float64 cross_entropy with probability targets (and its
+    label smoothing, which mixes the targets with the uniform distribution),
+    and its autograd, as an independent library special case; targets need
+    not sum to 1."""
+    torch = __import__("torch")
+    import torch.nn.functional as F
+    rng = np.random.default_rng(32)
+    for normalised in (True, False):
+        z, t = _soft_draw(rng, 7, 11, normalised)
+        g = rng.standard_normal(7)
+        for eps in (0.0, 0.25):
+            zt = torch.tensor(z, dtype=torch.float64, requires_grad=True)
+            ref = F.cross_entropy(zt, torch.tensor(t), reduction="none", label_smoothing=eps)
+            (ref * torch.tensor(g)).sum().backward()
+            loss, _ = orc.ce_soft_forward(z, t, eps)
+            np.testing.assert_allclose(loss, ref.detach().numpy(), rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(orc.ce_soft_backward(z, t, g, eps), zt.grad.numpy(),
+                                       rtol=1e-11, atol=1e-14)
+
+
+def pin_soft_closed_forms(orc):
+    """Equal logits against any distribution: loss = log V (t sums to 1).
+    Two logits [x, 0] against [1, 0]: log(1 + e^-x); against [a, 1-a] on
+    equal logits: log 2. Uniform targets with eps keep the loss."""
+    V = 10
+    t = np.random.default_rng(33).random((1, V)); t /= t.sum()
+    for c in (0.0, 1e4, 1e8):
+        loss, lse = orc.ce_soft_forward(np.full((1, V), c), t)
+        assert abs(loss[0] - math.log(V)) <= 1e-12 * math.log(V)
+        assert abs(lse[0] - (c + math.log(V))) <= 1e-15 * max(1.0, abs(c))
+    for x in (0.5, 3.0, -2.0):
+        loss, _ = orc.ce_soft_forward(np.array([[x, 0.0]]), np.array([[1.0, 0.0]]))
+        assert abs(loss[0] - math.log1p(math.exp(-x))) <= 1e-15
+    loss, _ = orc.ce_soft_forward(np.array([[5.0, 5.0]]), np.array([[0.3, 0.7]]))
+    assert abs(loss[0] - math.log(2.0)) <= 1e-15
+    z = np.array([[1.0, -2.0, 0.5, 3.0]])
+    u = np.full((1, 4), 0.25)
+    assert abs(orc.ce_soft_forward(z, u, 0.4)[0][0] - orc.ce_soft_forward(z, u, 0.0)[0][0]) <= 1e-15
+
+
+def pin_soft_grad_rows_sum_to_zero_and_shift(orc):
+    """Each gradient row sums to g (T' - T') = 0; shifting a row by c leaves
+    the loss unchanged for any targets (inputs on a 1/64 grid, so the shift
+    is exact)."""
+    rng = np.random.default_rng(34)
+    z = rng.integers(-256, 256, size=(6, 17)) / 64.0
+    t = rng.random((6, 17)) * 2 - 0.5
+    g = rng.standard_normal(6)
+    for eps in (0.0, 0.1):
+        dz = orc.ce_soft_backward(z, t, g, eps)
+        assert np.abs(dz.sum(1)).max() <= 1e-13 * (np.abs(dz).max() + 1)
+        l0, _ = orc.ce_soft_forward(z, t, eps)
+        l1, _ = orc.ce_soft_forward(z + 1024.0, t, eps)
+        np.testing.assert_allclose(l1, l0, rtol=1e-12, atol=1e-12)
+
+
+def pin_soft_finite_differences(orc):
+    """Central differences of sum_i g_i loss_i with respect to z."""
+    rng = np.random.default_rng(35)
+    z, t = _soft_draw(rng, 3, 6, normalised=False)
+    g = rng.standard_normal(3)
+    h = 1e-6
+    for eps in (0.0, 0.2):
+        dz = orc.ce_soft_backward(z, t, g, eps)
+        fd = np.zeros_like(z)
+        for idx in np.ndindex(z.shape):
+            zp = z.copy(); zp[idx] += h
+            zm = z.copy(); zm[idx] -= h
+            fd[idx] = (orc.ce_soft_forward(zp, t, eps)[0] @ g - orc.ce_soft_forward(zm, t, eps)[0] @ g) / (2 * h)
+        np.testing.assert_allclose(dz, fd, rtol=0, atol=1e-8)
+
+
+def pin_soft_nonfinite(orc):
+    """A -inf logit with zero target mass contributes nothing (0 log 0 = 0);
+    with target mass the loss is +inf; NaN rows and all -inf rows give NaN
+    losses and NaN gradient rows, with lse NaN and -inf."""
+    z = np.array([[1.0, -np.inf, 0.5], [1.0, -np.inf, 0.5], [1.0, np.nan, 0.5],
+                  [-np.inf, -np.inf, -np.inf]])
+    t = np.array([[0.5, 0.0, 0.5], [0.5, 0.25, 0.25], [0.3, 0.3, 0.4], [0.2, 0.3, 0.5]])
+    loss, lse = orc.ce_soft_forward(z, t)
+    ref0 = 0.5 * (math.log(math.e + math.exp(0.5)) - 1.0) + 0.5 * (math.log(math.e + math.exp(0.5)) - 0.5)
+    assert abs(loss[0] - ref0) <= 1e-15
+    assert loss[1] == math.inf
+    assert math.isnan(loss[2]) and math.isnan(lse[2])
+    assert math.isnan(loss[3]) and lse[3] == -math.inf
+    dz = orc.ce_soft_backward(z, t, 1.0)
+    assert np.isfinite(dz[:2]).all() and dz[0, 1] == 0.0
+    assert np.isnan(dz[2:]).all()
+
+
 # Ordered: cheap first. The planted-mistake test runs every entry.
 BATTERY = [
     pin_pr4188_printed_values,
@@ -328,4 +450,10 @@ BATTERY = [
     pin_finite_differences,
     pin_linear_vs_numpy,
     pin_linear_finite_differences,
+    pin_soft_onehot_matches_hard,
+    pin_soft_closed_forms,
+    pin_soft_grad_rows_sum_to_zero_and_shift,
+    pin_soft_nonfinite,
+    pin_soft_torch_float64,
+    pin_soft_finite_differences,
 ]

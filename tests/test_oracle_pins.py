@@ -71,6 +71,15 @@ MUTANTS = [
     ("dH contracts with H", "acc += G[i * V + j] * (double)W[j * D + d];\n            dH",
      "acc += G[i * V + j] * (double)H[i * D + d];\n            dH"),
     ("dh rows sign", "out[d] += gij * (double)w[d];", "out[d] -= gij * (double)w[d];"),
+    ("soft lse drops m", "*lse = m + L;", "*lse = L;"),
+    ("soft exp unshifted", "s += exp(z[j] - m);\n    const double L", "s += exp(z[j]);\n    const double L"),
+    ("soft loss sign", "l += tj * (L - (z[j] - m));", "l += tj * (L + (z[j] - m));"),
+    ("soft forward unsmoothed", "eps / (double)V;\n        if (tj", "0.0;\n        if (tj"),
+    ("soft zero-mass terms kept", "if (tj != 0.0) l += ", "l += "),
+    ("soft grad drops T", "d[j] = g[i] * (p * T - tj);", "d[j] = g[i] * (p - tj);"),
+    ("soft grad drops g", "d[j] = g[i] * (p * T - tj);", "d[j] = (p * T - tj);"),
+    ("soft grad unsmoothed target", "eps / (double)V;\n            d[j]", "0.0;\n            d[j]"),
+    ("soft grad unnormalised", "const double p = exp(zr[j] - m) / s;", "const double p = exp(zr[j] - m);"),
 ]
 
 
