@@ -169,6 +169,44 @@ ce_status ce_forward_backward(const void* logits, ce_dtype dt, ce_layout lg,
                               void* workspace, size_t ws_bytes, void* cuda_stream);
 
 /* ------------------------------------------------------------------------ *
+ * Probability (soft) targets. Source: MLX PR #4188, "Shift by the max in
+ * cross_entropy" (the loss is the row's log-sum-exp minus the
+ * target-weighted logits, assembled from values shifted by the row max).
+ * With a target distribution t per row and label smoothing eps (which mixes
+ * t with the uniform distribution: t' = (1-eps) t + eps/V):
+ *     loss_i = sum_j t'_ij (lse_i - z_ij),
+ *     dz_ij  = g_i (p_ij T'_i - t'_ij),   T'_i = sum_j t'_ij = (1-eps) T_i + eps,
+ * which is lse - sum_j t_j z_j and p - t when the rows of t sum to 1.
+ * t is used as given (not renormalised). A class whose t'_ij is 0 adds
+ * nothing, even at z_ij = -inf. NaN in a row, or a row of z that is all -inf,
+ * gives a NaN loss and a NaN gradient row. There is no ignore_index.
+ * Logits in f32, bf16 or f16; targets in the logits' dtype or f32 (else
+ * CE_ENOTSUP), N x V through their own layout `tl` (all four fields used).
+ * Each row of logits and of targets is read once per call; rows are not split
+ * across CTAs, so the calls want at least a few hundred rows to fill the GPU.
+ * ------------------------------------------------------------------------ */
+
+/* Forward: loss, lse (and lse_lo, as ce_forward; nullable) and, when
+ * target_sum is not NULL, T_i = sum_j t_ij per row (N floats) for the
+ * backward. No workspace. */
+ce_status ce_soft_forward(const void* logits, ce_dtype dt, ce_layout lg, int64_t N, int64_t V,
+                          const void* target_probs, ce_dtype tdt, ce_layout tl,
+                          float label_smoothing, float* loss, float* lse, float* lse_lo,
+                          float* target_sum, void* cuda_stream);
+
+/* Backward (VJP of sum_i g_i loss_i): dz as above from the saved lse (and
+ * lse_lo) and target_sum; target_sum NULL means every row of t sums to 1.
+ * grad_out, grad_stride and dlogits (dtype ddt: the logits' dtype or f32;
+ * in place on the logits allowed, same pointer, dtype and layout) as for
+ * ce_backward. */
+ce_status ce_soft_backward(const float* grad_out, int64_t grad_stride,
+                           const void* logits, ce_dtype dt, ce_layout lg, int64_t N, int64_t V,
+                           const void* target_probs, ce_dtype tdt, ce_layout tl,
+                           const float* lse, const float* lse_lo, const float* target_sum,
+                           float label_smoothing, void* dlogits, ce_dtype ddt, ce_layout dl,
+                           void* cuda_stream);
+
+/* ------------------------------------------------------------------------ *
  * Fused-linear cross-entropy: logits Z = H W^T are never stored.
  * Source: Ineshin, "A fused linear cross-entropy forward kernel for Apple
  * GPUs", section 1 (Z = H W^T streamed over vocabulary tiles into the running

@@ -25,7 +25,8 @@ STATUS = {0: "CE_OK", 1: "CE_EINVAL", 2: "CE_EALIAS", 3: "CE_EWORKSPACE", 4: "CE
           5: "CE_ETARGET", 6: "CE_ENOTSUP"}
 EXPORTED = ["ce_workspace_size", "ce_forward", "ce_backward", "linear_ce_workspace_size",
             "linear_ce_forward", "linear_ce_backward_workspace_size", "linear_ce_backward",
-            "ce_get_error", "ce_status_string", "ce_forward_noalloc", "ce_forward_backward"]
+            "ce_get_error", "ce_status_string", "ce_forward_noalloc", "ce_forward_backward",
+            "ce_soft_forward", "ce_soft_backward"]
 NOALLOC_SCRATCH_BYTES = 64 << 10
 
 
@@ -78,6 +79,12 @@ def lib() -> ctypes.CDLL:
                                           ce_layout, f32, i64, vp, i64, vp, vp, vp, vp, vp,
                                           ctypes.c_int, ce_layout, vp, sz, vp]
         L.ce_forward_backward.restype = ctypes.c_int
+        L.ce_soft_forward.argtypes = [vp, ctypes.c_int, ce_layout, i64, i64, vp, ctypes.c_int, ce_layout,
+                                      f32, vp, vp, vp, vp, vp]
+        L.ce_soft_forward.restype = ctypes.c_int
+        L.ce_soft_backward.argtypes = [vp, i64, vp, ctypes.c_int, ce_layout, i64, i64, vp, ctypes.c_int,
+                                       ce_layout, vp, vp, vp, f32, vp, ctypes.c_int, ce_layout, vp]
+        L.ce_soft_backward.restype = ctypes.c_int
         L.ce_get_error.argtypes = [vp]
         L.ce_get_error.restype = ctypes.c_int
         L.ce_status_string.argtypes = [ctypes.c_int]
@@ -271,6 +278,76 @@ def ce_backward(grad_out, logits, targets, lse, lse_lo=None, label_smoothing: fl
                                float(label_smoothing), int(ignore_index), _ptr(dlogits),
                                _dtype_code(dlogits), dl, _stream(stream))
     _check(st, "ce_backward")
+    return dlogits
+
+
+class SoftResult(NamedTuple):
+    loss: object
+    lse: object
+    lse_lo: object
+    target_sum: object
+
+
+def _grad_view(torch, grad_out, N):
+    if grad_out.dtype != torch.float32:
+        raise TypeError("grad_out must be float32")
+    if grad_out.numel() == 1:
+        return grad_out, 0
+    if grad_out.numel() != N:
+        raise ValueError("grad_out must hold one value per row or a single value")
+    gflat = grad_out.reshape(-1) if grad_out.dim() != 1 else grad_out
+    if gflat.data_ptr() != grad_out.data_ptr():
+        raise ValueError("grad_out must be a view over its storage")
+    return gflat, gflat.stride(0)
+
+
+def ce_soft_forward(logits, target_probs, label_smoothing: float = 0.0, *,
+                    return_target_sum: bool = True, stream=None) -> SoftResult:
+    """Cross-entropy against probability targets: loss_i = sum_j t'_ij
+    (lse_i - z_ij) with t' = (1-eps) t + eps/V. target_probs has the shape of
+    logits (any strides), dtype of the logits or float32. Also returns lse,
+    lse_lo and (if asked) the per-row sums of target_probs for the backward."""
+    torch = _torch()
+    _require_cuda(logits, target_probs)
+    N, lg = row_layout(logits, True)
+    Nt, tl = row_layout(target_probs, True)
+    if Nt != N or target_probs.shape[-1] != logits.shape[-1]:
+        raise ValueError("target_probs must have the shape of logits")
+    V = logits.shape[-1]
+    dev = logits.device
+    loss, lse, lse_lo = (torch.empty(N, dtype=torch.float32, device=dev) for _ in range(3))
+    tsum = torch.empty(N, dtype=torch.float32, device=dev) if return_target_sum else None
+    with torch.cuda.device(dev):
+        st = lib().ce_soft_forward(_ptr(logits), _dtype_code(logits), lg, N, V, _ptr(target_probs),
+                                   _dtype_code(target_probs), tl, float(label_smoothing), _ptr(loss),
+                                   _ptr(lse), _ptr(lse_lo), _ptr(tsum), _stream(stream))
+    _check(st, "ce_soft_forward")
+    return SoftResult(loss, lse, lse_lo, tsum)
+
+
+def ce_soft_backward(grad_out, logits, target_probs, lse, lse_lo=None, target_sum=None,
+                     label_smoothing: float = 0.0, *, dlogits=None, out_dtype=None, stream=None):
+    """dlogits = g (softmax T' - t'), T' = (1-eps) T + eps with T the row sums
+    of target_probs (target_sum from ce_soft_forward; None: rows sum to 1)."""
+    torch = _torch()
+    _require_cuda(grad_out, logits, target_probs, lse, lse_lo, target_sum, dlogits)
+    N, lg = row_layout(logits, True)
+    Nt, tl = row_layout(target_probs, True)
+    if Nt != N or target_probs.shape[-1] != logits.shape[-1]:
+        raise ValueError("target_probs must have the shape of logits")
+    V = logits.shape[-1]
+    grad_out, g_stride = _grad_view(torch, grad_out, N)
+    if dlogits is None:
+        dlogits = torch.empty(logits.shape, dtype=out_dtype or logits.dtype, device=logits.device)
+    Nd, dl = row_layout(dlogits, True)
+    if Nd != N or dlogits.shape[-1] != V:
+        raise ValueError("dlogits must have the shape of logits")
+    with torch.cuda.device(logits.device):
+        st = lib().ce_soft_backward(_ptr(grad_out), g_stride, _ptr(logits), _dtype_code(logits), lg, N, V,
+                                    _ptr(target_probs), _dtype_code(target_probs), tl, _ptr(lse),
+                                    _ptr(lse_lo), _ptr(target_sum), float(label_smoothing),
+                                    _ptr(dlogits), _dtype_code(dlogits), dl, _stream(stream))
+    _check(st, "ce_soft_backward")
     return dlogits
 
 

@@ -362,6 +362,118 @@ ce_status ce_backward(const float* grad_out, int64_t grad_stride, const void* lo
     return e == cudaSuccess ? CE_OK : CE_ECUDA;
 }
 
+// ---- probability (soft) targets -------------------------------------------------
+static SoftPlan plan_soft(int64_t N, int64_t V, int esz, bool vec_ok, int sms) {
+    SoftPlan p{};
+    p.vec = vec_ok ? 16 / esz : 1;
+    const int U = p.vec == 1 ? 8 : (esz == 4 ? 4 : 2);
+    const int64_t nvec = V / p.vec;
+    int G = 1;
+    while (G < 32 && nvec > (int64_t)U * G) G *= 2;
+    p.G = G;
+    const int64_t rows_per_block = 8 * (32 / G);
+    const int64_t want = (N + rows_per_block - 1) / rows_per_block;
+    const int64_t cap = (int64_t)sms * 16;
+    p.grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
+    return p;
+}
+
+static bool soft_dtypes_ok(ce_dtype dt, ce_dtype tdt) {
+    if (dt != CE_F32 && dt != CE_BF16 && dt != CE_F16) return false;
+    return tdt == dt || tdt == CE_F32;
+}
+
+ce_status ce_soft_forward(const void* logits, ce_dtype dt, ce_layout lg, int64_t N, int64_t V,
+                          const void* target_probs, ce_dtype tdt, ce_layout tl,
+                          float label_smoothing, float* loss, float* lse, float* lse_lo,
+                          float* target_sum, void* cuda_stream) {
+    if (N < 0 || V < 1 || V > INT32_MAX) return CE_EINVAL;
+    if (!soft_dtypes_ok(dt, tdt)) return CE_ENOTSUP;
+    if (!(label_smoothing >= 0.f && label_smoothing <= 1.f)) return CE_EINVAL;
+    if (N == 0) return CE_OK;
+    if (!logits || !target_probs || !loss || !lse) return CE_EINVAL;
+    if (!layout_ok(lg) || !layout_ok(tl)) return CE_EINVAL;
+    const int esz = elem_size(dt), tsz = elem_size(tdt);
+    const Layout L = to_layout(lg), T = to_layout(tl);
+    const Extent ez = layout_extent(logits, L, N, V, esz);
+    const Extent et = layout_extent(target_probs, T, N, V, tsz);
+    Extent outs[4];
+    int nout = 0;
+    outs[nout++] = flat_extent(loss, N, 4);
+    outs[nout++] = flat_extent(lse, N, 4);
+    if (lse_lo) outs[nout++] = flat_extent(lse_lo, N, 4);
+    if (target_sum) outs[nout++] = flat_extent(target_sum, N, 4);
+    for (int i = 0; i < nout; ++i) {
+        if (overlap(outs[i], ez) || overlap(outs[i], et)) return CE_EALIAS;
+        for (int j = 0; j < i; ++j)
+            if (overlap(outs[i], outs[j])) return CE_EALIAS;
+    }
+    const bool vec_ok = vectorizable(logits, L, N, esz) && vectorizable(target_probs, T, N, tsz);
+    SoftPlan p = plan_soft(N, V, esz, vec_ok, device_sms(0));
+    SoftArgs a{};
+    a.z = logits;
+    a.t = target_probs;
+    a.N = N;
+    a.V = V;
+    a.eps = label_smoothing;
+    a.loss = loss;
+    a.lse = lse;
+    a.lse_lo = lse_lo;
+    a.tsum = target_sum;
+    a.lz = L;
+    a.lt = T;
+    cudaError_t e = launch_soft_forward(p, a, (int)dt, (int)tdt, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? CE_OK : CE_ECUDA;
+}
+
+ce_status ce_soft_backward(const float* grad_out, int64_t grad_stride, const void* logits, ce_dtype dt,
+                           ce_layout lg, int64_t N, int64_t V, const void* target_probs, ce_dtype tdt,
+                           ce_layout tl, const float* lse, const float* lse_lo, const float* target_sum,
+                           float label_smoothing, void* dlogits, ce_dtype ddt, ce_layout dl,
+                           void* cuda_stream) {
+    if (N < 0 || V < 1 || V > INT32_MAX) return CE_EINVAL;
+    if (!soft_dtypes_ok(dt, tdt)) return CE_ENOTSUP;
+    if (ddt != CE_F32 && ddt != dt) return CE_ENOTSUP;
+    if (!(label_smoothing >= 0.f && label_smoothing <= 1.f)) return CE_EINVAL;
+    if (N == 0) return CE_OK;
+    if (!grad_out || !logits || !target_probs || !lse || !dlogits) return CE_EINVAL;
+    if (!layout_ok(lg) || !layout_ok(tl) || !layout_ok(dl)) return CE_EINVAL;
+    const int esz = elem_size(dt), tsz = elem_size(tdt), dsz = elem_size(ddt);
+    const Layout L = to_layout(lg), T = to_layout(tl), D = to_layout(dl);
+    const Extent ez = layout_extent(logits, L, N, V, esz);
+    const Extent et = layout_extent(target_probs, T, N, V, tsz);
+    const Extent ed = layout_extent(dlogits, D, N, V, dsz);
+    const Extent eg = grad_stride == 0 ? flat_extent(grad_out, 1, 4)
+                                       : layout_extent(grad_out, Layout{N, 0, grad_stride, 0}, N, 1, 4);
+    const bool in_place = dlogits == logits && ddt == dt && L.inner == D.inner &&
+                          L.s_outer == D.s_outer && L.s_inner == D.s_inner && L.s_col == D.s_col;
+    if (!in_place && overlap(ed, ez)) return CE_EALIAS;
+    if (overlap(ed, et) || overlap(ed, eg) || overlap(ed, flat_extent(lse, N, 4))) return CE_EALIAS;
+    if (lse_lo && overlap(ed, flat_extent(lse_lo, N, 4))) return CE_EALIAS;
+    if (target_sum && overlap(ed, flat_extent(target_sum, N, 4))) return CE_EALIAS;
+    const bool vec_ok = vectorizable(logits, L, N, esz) && vectorizable(target_probs, T, N, tsz) &&
+                        vectorizable(dlogits, D, N, dsz);
+    SoftPlan p = plan_soft(N, V, esz, vec_ok, device_sms(0));
+    SoftArgs a{};
+    a.z = logits;
+    a.t = target_probs;
+    a.N = N;
+    a.V = V;
+    a.eps = label_smoothing;
+    a.lse = const_cast<float*>(lse);
+    a.lse_lo = const_cast<float*>(lse_lo);
+    a.tsum = const_cast<float*>(target_sum);
+    a.g = grad_out;
+    a.g_stride = grad_stride;
+    a.dz = dlogits;
+    a.lz = L;
+    a.lt = T;
+    a.ld = D;
+    cudaError_t e = launch_soft_backward(p, a, (int)dt, (int)tdt, (int)ddt,
+                                         static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? CE_OK : CE_ECUDA;
+}
+
 ce_status ce_forward_backward(const void* logits, ce_dtype dt, ce_layout lg, int64_t N, int64_t V,
                               const void* targets, ce_index_dtype tdt, ce_layout tg,
                               float label_smoothing, int64_t ignore_index, const float* grad_out,

@@ -116,4 +116,31 @@ struct SmemRowPlan {
 cudaError_t launch_fused_smem(const SmemRowPlan& p, const FusedArgs& a, int dt_in, int dt_out,
                               cudaStream_t s);
 
+// ---- probability (soft) targets ---------------------------------------------
+struct SoftArgs {
+    const void* z;
+    const void* t;
+    int64_t N, V;
+    float eps;
+    float* loss;
+    float* lse;
+    float* lse_lo;
+    float* tsum;        // forward: sum_j t_j per row (nullable)
+    const float* g;     // backward
+    int64_t g_stride;
+    void* dz;
+    Layout lz, lt, ld;
+};
+
+struct SoftPlan {
+    int vec;
+    int G;
+    int grid;
+};
+
+cudaError_t launch_soft_forward(const SoftPlan& p, const SoftArgs& a, int dz_t, int dt_t,
+                                cudaStream_t s);
+cudaError_t launch_soft_backward(const SoftPlan& p, const SoftArgs& a, int dz_t, int dt_t, int do_t,
+                                 cudaStream_t s);
+
 }  // namespace ceb

@@ -187,3 +187,30 @@ def test_out_tensors_validated():
             ce._row_outputs(5, torch.device("cpu"), False, bad)
     with pytest.raises(ValueError):
         ce._row_outputs(5, torch.device("cpu"), True, good)  # argmax requested, none given
+
+
+def soft_fwd(L, z=Z, dt=0, N=8, V=16, t=T, tdt=0, tl=None, eps=0.0, loss=OUT, lse=OUT + 4096,
+             lse_lo=None, tsum=None):
+    tl = tl or lay(N, V)
+    return L.ce_soft_forward(z, dt, lay(N, V), N, V, t, tdt, tl, eps, loss, lse, lse_lo, tsum, None)
+
+
+def soft_bwd(L, g=OUT + 8192, z=Z, dt=0, N=8, V=16, t=T, tdt=0, lse=OUT, tsum=None, eps=0.0,
+             dz=0x40000000, ddt=0):
+    return L.ce_soft_backward(g, 0, z, dt, lay(N, V), N, V, t, tdt, lay(N, V), lse, None, tsum, eps,
+                              dz, ddt, lay(N, V), None)
+
+
+def test_soft_targets_reject_bad_arguments_and_aliasing(L):
+    assert soft_fwd(L, N=-1) == 1
+    assert soft_fwd(L, eps=2.0) == 1
+    assert soft_fwd(L, t=None) == 1
+    assert soft_fwd(L, dt=1, tdt=2) == 6      # f16 targets for bf16 logits: not supported
+    assert soft_fwd(L, dt=0, tdt=1) == 6      # bf16 targets for f32 logits: not supported
+    assert soft_fwd(L, N=0, z=None, t=None, loss=None, lse=None) == 0
+    assert soft_fwd(L, loss=T + 32) == 2      # loss over the targets
+    assert soft_fwd(L, tsum=OUT + 8) == 2     # target sums over loss
+    assert soft_bwd(L, ddt=2) == 6            # f16 gradient of f32 logits
+    assert soft_bwd(L, dz=T + 64) == 2        # gradient over the targets
+    assert soft_bwd(L, dz=OUT) == 2           # gradient over lse
+    assert soft_bwd(L, g=None) == 1
