@@ -391,6 +391,114 @@ def bench_rows(args, rk):
     return out, (z32, y, eps, kind)
 
 
+# -- probability (soft) targets --------------------------------------------------------------
+SOFT_DESC = ("8192 x 32000 bf16 logits ~N(0, std 2) against bf16 target distributions "
+             "(normalised U[0,1) draws), bf16 dlogits; forward + backward")
+
+
+def soft_inputs(seed: int, N: int = 8192, V: int = 32000):
+    rng = np.random.default_rng(seed)
+    z, _ = wl.encode(rng.standard_normal((N, V), dtype=np.float32) * 2, "bf16")
+    t = rng.random((N, V), dtype=np.float32)
+    t /= t.sum(1, keepdims=True)
+    t, _ = wl.encode(t, "bf16")
+    return z, t
+
+
+def bench_soft(args, rk):
+    import torch
+    import softmax_cross_entropy_lse_b200 as ce
+    world = rk.world
+    z, t = soft_inputs(rk.rank)
+    if args.rows:
+        z, t = z[:args.rows], t[:args.rows]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    z_h = torch.from_numpy(np.ascontiguousarray(z).view(np.int16)).view(torch.bfloat16)
+    t_h = torch.from_numpy(np.ascontiguousarray(t).view(np.int16)).view(torch.bfloat16)
+    z_d, t_d = z_h.to(dev), t_h.to(dev)
+    N, V = z_d.shape
+    g = torch.full((1,), 1.0 / N, dtype=torch.float32, device=dev)
+    dz = torch.empty_like(z_d)
+    stream = torch.cuda.current_stream()
+    fwd_bytes = N * V * 4 + 16 * N
+    bwd_bytes = N * V * 6 + 16 * N
+    step_bytes = fwd_bytes + bwd_bytes
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        r = ce.ce_soft_forward(z_d, t_d)
+        if ev is not None:
+            ev[1].record(stream)
+        ce.ce_soft_backward(g, z_d, t_d, r.lse, r.lse_lo, r.target_sum, dlogits=dz)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        sharding.barrier(rk)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        sharding.barrier(rk)
+    ms = sharding.max_over_ranks(rk, t0.elapsed_time(t1))
+    fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    # end to end: logits and targets copied in from pinned host memory, loss out
+    z_pin, t_pin = z_h.pin_memory(), t_h.pin_memory()
+    loss_h = torch.empty(N, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        z_d.copy_(z_pin, non_blocking=True)
+        t_d.copy_(t_pin, non_blocking=True)
+        r = ce.ce_soft_forward(z_d, t_d)
+        ce.ce_soft_backward(g, z_d, t_d, r.lse, r.lse_lo, r.target_sum, dlogits=dz)
+        loss_h.copy_(r.loss, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    sharding.barrier(rk)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(3):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sharding.max_over_ranks(rk, a.elapsed_time(b)) / 3
+    peak_hbm, _, _, peak_src = load_peaks()
+    dom, dom_ms, dom_bytes = ("backward", bwd_ms, bwd_bytes) if bwd_ms >= fwd_ms else \
+        ("forward", fwd_ms, fwd_bytes)
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    out = {
+        "metric": METRIC, "value": round(world * step_bytes * args.steps / (ms * 1e-3) / 1e9, 2),
+        "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "fwd_GBs": round(fwd_bytes / (fwd_ms * 1e-3) / 1e9, 2),
+        "bwd_GBs": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9, 2),
+        "config": {"workload": f"soft: {SOFT_DESC}", "rows": N, "classes": V,
+                   "bytes_per_step": step_bytes, "l2": "inputs larger than L2",
+                   "parallelism": f"rows sharded over {world} rank(s), no data-path collective"},
+        "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": 2 * N * V * 2, "d2h_bytes_per_step": 4 * N},
+        "gpu_launches": 2 * args.steps,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 2), "peak": peak_hbm,
+                     "unit": "GB/s", "frac": round(achieved / peak_hbm, 4), "traffic": None,
+                     "peak_source": peak_src, "algorithmic_bytes_per_launch": dom_bytes},
+    }
+    clocks = clk.summary()
+    if clocks:
+        out["clocks"] = clocks
+    return out, None
+
+
 # -- fused-linear workload -------------------------------------------------------------------
 def bench_linear(args, rk):
     import torch
@@ -564,6 +672,33 @@ class OracleLinear:
         return int(max(n, (seconds / per_row) // n * n))
 
 
+class OracleSoft(OracleRows):
+    """The float64 oracle for probability targets (forward + backward)."""
+
+    def __init__(self):
+        import oracle
+        self.orc = oracle.get()
+        z, t = soft_inputs(0)
+        self.z32 = wl.f32_from_bf16_bits(z)
+        self.t32 = wl.f32_from_bf16_bits(t)
+        self.N, self.V = self.z32.shape
+        self.bytes_per_row = 5 * self.V * 2 + 32
+        self.cursor = 0
+
+    def run(self, rows: int) -> None:
+        done = 0
+        chunk = max(1, int(5e7 // self.V))
+        while done < rows:
+            lo = self.cursor % self.N
+            n = min(chunk, rows - done, self.N - lo)
+            zc = self.z32[lo:lo + n].astype(np.float64)
+            tc = self.t32[lo:lo + n].astype(np.float64)
+            self.orc.ce_soft_forward(zc, tc)
+            self.orc.ce_soft_backward(zc, tc, 1.0)
+            self.cursor += n
+            done += n
+
+
 def oracle_baseline(workload, seconds: float, host=None):
     """(value, unit, cores, sample) of the oracle timed for about `seconds`."""
     if workload == "c5":
@@ -574,7 +709,7 @@ def oracle_baseline(workload, seconds: float, host=None):
         dt = time.perf_counter() - t
         return (rows * o.flop_per_row / dt / 1e12, "TFLOP/s", o.orc.num_threads(),
                 f"{rows} of 8192 rows of c5 (loss, lse and dH rows), {dt:.1f} s")
-    o = OracleRows(workload, host)
+    o = OracleSoft() if workload == "soft" else OracleRows(workload, host)
     rows = min(o.rows_for(seconds), 50 * o.N)
     t = time.perf_counter()
     o.run(rows)
@@ -592,7 +727,7 @@ def run_reference(args):
         o = OracleLinear()
         unit, per_row = "TFLOP/s", o.flop_per_row / 1e12
     else:
-        o = OracleRows(args.workload)
+        o = OracleSoft() if args.workload == "soft" else OracleRows(args.workload)
         unit, per_row = "GB/s", o.bytes_per_row / 1e9
     # each step a bounded sample, so the whole run stays within about two minutes
     step_s = min(2.0, 120.0 / (args.steps + args.warmup))
@@ -626,7 +761,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="c2", choices=sorted(ROW_WORKLOADS) + ["c5"])
+    ap.add_argument("--workload", default="c2", choices=sorted(ROW_WORKLOADS) + ["c5", "soft"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rows", type=int, default=0,
@@ -645,6 +780,8 @@ def main():
     rk = dist_setup(args.gpus)
     if args.workload == "c5":
         out, host = bench_linear(args, rk)
+    elif args.workload == "soft":
+        out, host = bench_soft(args, rk)
     else:
         out, host = bench_rows(args, rk)
     if rk.rank == 0 and rk.world == 1 and not args.no_cpu_baseline:

@@ -363,10 +363,11 @@ ce_status ce_backward(const float* grad_out, int64_t grad_stride, const void* lo
 }
 
 // ---- probability (soft) targets -------------------------------------------------
-static SoftPlan plan_soft(int64_t N, int64_t V, int esz, bool vec_ok, int sms) {
+static SoftPlan plan_soft(int64_t N, int64_t V, int esz, int tsz, bool vec_ok, int sms) {
     SoftPlan p{};
     p.vec = vec_ok ? 16 / esz : 1;
-    const int U = p.vec == 1 ? 8 : (esz == 4 ? 4 : 2);
+    // vectors per lane per step, as the kernels take them
+    const int U = p.vec == 1 ? 8 : (tsz > esz ? 2 : 4);
     const int64_t nvec = V / p.vec;
     int G = 1;
     while (G < 32 && nvec > (int64_t)U * G) G *= 2;
@@ -409,7 +410,7 @@ ce_status ce_soft_forward(const void* logits, ce_dtype dt, ce_layout lg, int64_t
             if (overlap(outs[i], outs[j])) return CE_EALIAS;
     }
     const bool vec_ok = vectorizable(logits, L, N, esz) && vectorizable(target_probs, T, N, tsz);
-    SoftPlan p = plan_soft(N, V, esz, vec_ok, device_sms(0));
+    SoftPlan p = plan_soft(N, V, esz, tsz, vec_ok, device_sms(0));
     SoftArgs a{};
     a.z = logits;
     a.t = target_probs;
@@ -453,7 +454,7 @@ ce_status ce_soft_backward(const float* grad_out, int64_t grad_stride, const voi
     if (target_sum && overlap(ed, flat_extent(target_sum, N, 4))) return CE_EALIAS;
     const bool vec_ok = vectorizable(logits, L, N, esz) && vectorizable(target_probs, T, N, tsz) &&
                         vectorizable(dlogits, D, N, dsz);
-    SoftPlan p = plan_soft(N, V, esz, vec_ok, device_sms(0));
+    SoftPlan p = plan_soft(N, V, esz, tsz, vec_ok, device_sms(0));
     SoftArgs a{};
     a.z = logits;
     a.t = target_probs;

@@ -42,6 +42,36 @@ __device__ __forceinline__ void load_n(const T* p, int64_t col, int64_t s_col, f
     }
 }
 
+// VEC elements of T held as raw 16-byte words (VEC > 1) or one float (VEC =
+// 1) between the load and the use, so that many loads can be in flight in
+// few registers.
+template <typename T, int VEC>
+struct Raw {
+    static constexpr int W = VEC == 1 ? 1 : (int)(VEC * sizeof(T) / 16);
+    uint4 w[W];
+};
+
+template <typename T, int VEC>
+__device__ __forceinline__ void load_raw(const T* p, int64_t col, int64_t s_col, Raw<T, VEC>& r) {
+    if constexpr (VEC == 1) {
+        r.w[0].x = __float_as_uint(to_f32(p[col * s_col]));
+    } else {
+#pragma unroll
+        for (int w = 0; w < Raw<T, VEC>::W; ++w) r.w[w] = __ldcs(reinterpret_cast<const uint4*>(p + col) + w);
+    }
+}
+
+template <typename T, int VEC>
+__device__ __forceinline__ void unpack_raw(const Raw<T, VEC>& r, float (&out)[VEC]) {
+    if constexpr (VEC == 1) {
+        out[0] = __uint_as_float(r.w[0].x);
+    } else {
+        constexpr int PER = 16 / (int)sizeof(T);
+#pragma unroll
+        for (int w = 0; w < Raw<T, VEC>::W; ++w) unpack_words<T>(r.w[w], out + w * PER);
+    }
+}
+
 template <bool EPS>
 __device__ __forceinline__ void soft_rescale(SoftState& st, float mn) {
     if (st.m != mn) {
@@ -101,8 +131,8 @@ __device__ __forceinline__ void soft_group_reduce(SoftState& st) {
     }
 }
 
-template <typename TZ, typename TT, int VEC, int G, int U, bool EPS>
-__global__ void __launch_bounds__(256, 2) k_soft_fwd(SoftArgs a) {
+template <typename TZ, typename TT, int VEC, int G, int U, bool EPS, int MINB>
+__global__ void __launch_bounds__(256, MINB) k_soft_fwd(SoftArgs a) {
     const TZ* __restrict__ z = reinterpret_cast<const TZ*>(a.z);
     const TT* __restrict__ tg = reinterpret_cast<const TT*>(a.t);
     const int lane = threadIdx.x & 31;
@@ -125,20 +155,26 @@ __global__ void __launch_bounds__(256, 2) k_soft_fwd(SoftArgs a) {
             tr = tg + row_offset(a.lt, r, a.N);
         }
         for (int64_t vb = 0; vb < nvec; vb += (int64_t)G * U) {
-            float zv[U][VEC], tv[U][VEC];
+            Raw<TZ, VEC> rz[U];
+            Raw<TT, VEC> rt[U];
             bool ok[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int64_t vi = vb + u * G + gl;
                 ok[u] = active && vi < nvec;
                 if (ok[u]) {
-                    load_n<TZ, VEC>(zr, vi * VEC, a.lz.s_col, zv[u]);
-                    load_n<TT, VEC>(tr, vi * VEC, a.lt.s_col, tv[u]);
+                    load_raw<TZ, VEC>(zr, vi * VEC, a.lz.s_col, rz[u]);
+                    load_raw<TT, VEC>(tr, vi * VEC, a.lt.s_col, rt[u]);
                 }
             }
 #pragma unroll
-            for (int u = 0; u < U; ++u)
-                if (ok[u]) soft_fold<VEC, EPS>(st, zv[u], tv[u]);
+            for (int u = 0; u < U; ++u) {
+                if (!ok[u]) continue;
+                float zv[VEC], tv[VEC];
+                unpack_raw<TZ, VEC>(rz[u], zv);
+                unpack_raw<TT, VEC>(rt[u], tv);
+                soft_fold<VEC, EPS>(st, zv, tv);
+            }
         }
         if (active) {
             for (int q = gl; q < tail; q += G) {
@@ -172,8 +208,8 @@ __global__ void __launch_bounds__(256, 2) k_soft_fwd(SoftArgs a) {
     }
 }
 
-template <typename TZ, typename TT, typename TO, int VEC, int G, int U>
-__global__ void __launch_bounds__(256, 2) k_soft_bwd(SoftArgs a) {
+template <typename TZ, typename TT, typename TO, int VEC, int G, int U, int MINB>
+__global__ void __launch_bounds__(256, MINB) k_soft_bwd(SoftArgs a) {
     const TZ* z = reinterpret_cast<const TZ*>(a.z);
     const TT* __restrict__ tg = reinterpret_cast<const TT*>(a.t);
     TO* dz = reinterpret_cast<TO*>(a.dz);
@@ -198,25 +234,28 @@ __global__ void __launch_bounds__(256, 2) k_soft_bwd(SoftArgs a) {
         const float Tp = a.tsum ? (1.f - eps) * a.tsum[r] + eps : 1.f;
         const float gT = g * Tp, g1 = g * (1.f - eps), ge = g * eps_v;
         for (int64_t vb = gl; vb < nvec; vb += (int64_t)G * U) {
-            float zv[U][VEC], tv[U][VEC];
+            Raw<TZ, VEC> rz[U];
+            Raw<TT, VEC> rt[U];
             bool ok[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int64_t vi = vb + (int64_t)u * G;
                 ok[u] = vi < nvec;
                 if (ok[u]) {
-                    load_n<TZ, VEC>(zr, vi * VEC, a.lz.s_col, zv[u]);
-                    load_n<TT, VEC>(tr, vi * VEC, a.lt.s_col, tv[u]);
+                    load_raw<TZ, VEC>(zr, vi * VEC, a.lz.s_col, rz[u]);
+                    load_raw<TT, VEC>(tr, vi * VEC, a.lt.s_col, rt[u]);
                 }
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 if (!ok[u]) continue;
-                float o[VEC];
+                float zv[VEC], tv[VEC], o[VEC];
+                unpack_raw<TZ, VEC>(rz[u], zv);
+                unpack_raw<TT, VEC>(rt[u], tv);
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) {
-                    const float p = ex2(fmaf(zv[u][e] - hi, kLog2e, -c_lo));
-                    o[e] = fmaf(gT, p, -fmaf(g1, tv[u][e], ge));
+                    const float p = ex2(fmaf(zv[e] - hi, kLog2e, -c_lo));
+                    o[e] = fmaf(gT, p, -fmaf(g1, tv[e], ge));
                 }
                 store_vec<TO, VEC>(dr, (vb + (int64_t)u * G) * VEC, a.ld.s_col, o);
             }
@@ -233,12 +272,23 @@ __global__ void __launch_bounds__(256, 2) k_soft_bwd(SoftArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Vectors per lane per step and resident blocks: raw words keep four
+// vectors of logits and targets in flight per lane within a 64-register
+// budget (four blocks per SM; three for the backward of 16-bit logits,
+// whose eight-wide vectors need more registers); the scalar path keeps eight.
+// The planner's lane grouping uses the same U (plan_soft).
+template <typename TZ, typename TT, int VEC, bool BWD = false> struct SoftShape {
+    // float targets of 16-bit logits take twice the words: two vectors
+    static constexpr int U = VEC == 1 ? 8 : (sizeof(TT) > sizeof(TZ) ? 2 : 4);
+    static constexpr int MINB = VEC == 1 ? 2 : ((BWD && VEC == 8) ? 3 : 4);
+};
+
 template <typename TZ, typename TT, int VEC, bool EPS>
 static cudaError_t launch_soft_fwd_v(const SoftPlan& p, const SoftArgs& a, cudaStream_t s) {
-    constexpr int U = VEC == 1 ? 8 : (sizeof(TZ) == 4 ? 4 : 2);
+    constexpr int U = SoftShape<TZ, TT, VEC>::U, MB = SoftShape<TZ, TT, VEC>::MINB;
 #define CEB_SOFT(GG)                                                              \
     if (p.G == GG) {                                                              \
-        k_soft_fwd<TZ, TT, VEC, GG, U, EPS><<<p.grid, 256, 0, s>>>(a);            \
+        k_soft_fwd<TZ, TT, VEC, GG, U, EPS, MB><<<p.grid, 256, 0, s>>>(a);        \
         return cudaGetLastError();                                                \
     }
     CEB_SOFT(1) CEB_SOFT(2) CEB_SOFT(4) CEB_SOFT(8) CEB_SOFT(16) CEB_SOFT(32)
@@ -248,10 +298,10 @@ static cudaError_t launch_soft_fwd_v(const SoftPlan& p, const SoftArgs& a, cudaS
 
 template <typename TZ, typename TT, typename TO, int VEC>
 static cudaError_t launch_soft_bwd_v(const SoftPlan& p, const SoftArgs& a, cudaStream_t s) {
-    constexpr int U = VEC == 1 ? 8 : (sizeof(TZ) == 4 ? 4 : 2);
+    constexpr int U = SoftShape<TZ, TT, VEC, true>::U, MB = SoftShape<TZ, TT, VEC, true>::MINB;
 #define CEB_SOFT(GG)                                                              \
     if (p.G == GG) {                                                              \
-        k_soft_bwd<TZ, TT, TO, VEC, GG, U><<<p.grid, 256, 0, s>>>(a);             \
+        k_soft_bwd<TZ, TT, TO, VEC, GG, U, MB><<<p.grid, 256, 0, s>>>(a);         \
         return cudaGetLastError();                                                \
     }
     CEB_SOFT(1) CEB_SOFT(2) CEB_SOFT(4) CEB_SOFT(8) CEB_SOFT(16) CEB_SOFT(32)
