@@ -55,6 +55,8 @@ class Oracle:
                                              ctypes.c_double, _i64, _f64p, _f64p, _f64p]
         L.orc_ce_soft_forward.argtypes = [_f64p, _f64p, _i64, _i64, ctypes.c_double, _f64p, _f64p]
         L.orc_ce_soft_backward.argtypes = [_f64p, _f64p, _i64, _i64, _f64p, ctypes.c_double, _f64p]
+        L.orc_kl_forward.argtypes = [_f64p, _f64p, _i64, _i64, _f64p, _f64p, _f64p]
+        L.orc_kl_backward.argtypes = [_f64p, _f64p, _i64, _i64, _f64p, _f64p]
         L.orc_num_threads.restype = ctypes.c_int
 
     # -- helpers -----------------------------------------------------------
@@ -112,6 +114,30 @@ class Oracle:
         self.lib.orc_ce_soft_backward(self._p(z, _f64p), self._p(t, _f64p), N, V,
                                       self._p(g, _f64p), float(eps), self._p(dz, _f64p))
         return dz
+
+    # -- KL divergence of the student from the teacher ----------------------
+    def kl_forward(self, zq, zp):
+        """loss = sum_j p_j (log p_j - log q_j), lse of the student and of the
+        teacher (float64, N each); zq student, zp teacher logits (N, V)."""
+        zq = np.ascontiguousarray(zq, dtype=np.float64)
+        zp = np.ascontiguousarray(zp, dtype=np.float64)
+        N, V = zq.shape
+        assert zp.shape == (N, V)
+        loss, lq, lp = (np.empty(N, np.float64) for _ in range(3))
+        self.lib.orc_kl_forward(self._p(zq, _f64p), self._p(zp, _f64p), N, V, self._p(loss, _f64p),
+                                self._p(lq, _f64p), self._p(lp, _f64p))
+        return loss, lq, lp
+
+    def kl_backward(self, zq, zp, g):
+        """Gradient of sum_i g_i loss_i with respect to the student logits."""
+        zq = np.ascontiguousarray(zq, dtype=np.float64)
+        zp = np.ascontiguousarray(zp, dtype=np.float64)
+        N, V = zq.shape
+        g = np.ascontiguousarray(np.broadcast_to(np.asarray(g, np.float64), (N,)))
+        d = np.empty((N, V), np.float64)
+        self.lib.orc_kl_backward(self._p(zq, _f64p), self._p(zp, _f64p), N, V, self._p(g, _f64p),
+                                 self._p(d, _f64p))
+        return d
 
     # -- fused-linear cross-entropy ---------------------------------------
     def linear_ce_forward_rows(self, H, W, y, rows=None, eps: float = 0.0,

@@ -332,6 +332,74 @@ void orc_ce_soft_backward(const double* z, const double* t, int64_t N, int64_t V
     }
 }
 
+/* ---- KL divergence of a student distribution from a teacher's ------------
+ * "One barrier short" (Suryavanshi), the fused KL loss of mlx-lm: per row,
+ * with teacher logits zp and student logits zq over the same V classes,
+ *     p = softmax(zp), q = softmax(zq),
+ *     loss = sum_j p_j (log p_j - log q_j),
+ * and the gradient of sum_i g_i loss_i with respect to the student logits,
+ *     dzq_j = g (q_j - p_j).
+ * Readings where the pages are silent:
+ *   - a class with p_j = 0 (teacher logit -inf) adds nothing, even where
+ *     the student's is -inf too (0 log 0 = 0); a student -inf under teacher
+ *     mass makes the loss +inf.
+ *   - NaN in either row, or a row of either that is all -inf: loss NaN and
+ *     a NaN gradient row; each lse as for the cross-entropy (NaN, -inf). */
+static double row_lse(const double* z, int64_t V, double* m_out, double* s_out)
+{
+    double m = -INFINITY;
+    for (int64_t j = 0; j < V; ++j) {
+        if (isnan(z[j])) { *m_out = NAN; *s_out = NAN; return NAN; }
+        if (z[j] > m) m = z[j];
+    }
+    *m_out = m;
+    if (m == -INFINITY) { *s_out = 0.0; return -INFINITY; }
+    double s = 0.0;
+    for (int64_t j = 0; j < V; ++j) s += exp(z[j] - m);
+    *s_out = s;
+    return m + log(s);
+}
+
+void orc_kl_forward(const double* zq, const double* zp, int64_t N, int64_t V,
+                    double* loss, double* lse_q, double* lse_p)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i) {
+        const double* q = zq + i * V;
+        const double* p = zp + i * V;
+        double mq, sq, mp, sp;
+        lse_q[i] = row_lse(q, V, &mq, &sq);
+        lse_p[i] = row_lse(p, V, &mp, &sp);
+        if (!isfinite(lse_q[i]) || !isfinite(lse_p[i])) { loss[i] = NAN; continue; }
+        double l = 0.0;
+        for (int64_t j = 0; j < V; ++j) {
+            const double lp = p[j] - lse_p[i];
+            const double pj = exp(lp);
+            if (pj != 0.0) l += pj * (lp - (q[j] - lse_q[i]));
+        }
+        loss[i] = l;
+    }
+}
+
+void orc_kl_backward(const double* zq, const double* zp, int64_t N, int64_t V,
+                     const double* g, double* dzq)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i) {
+        const double* q = zq + i * V;
+        const double* p = zp + i * V;
+        double* d = dzq + i * V;
+        double mq, sq, mp, sp;
+        const double lq = row_lse(q, V, &mq, &sq);
+        const double lp = row_lse(p, V, &mp, &sp);
+        if (!isfinite(lq) || !isfinite(lp)) {
+            for (int64_t j = 0; j < V; ++j) d[j] = NAN;
+            continue;
+        }
+        for (int64_t j = 0; j < V; ++j) d[j] = g[i] * (exp(q[j] - lq) - exp(p[j] - lp));
+    }
+}
+
 /* Threads OpenMP will use, for reporting the CPU baseline's core count. */
 int orc_num_threads(void)
 {

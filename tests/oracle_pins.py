@@ -20,6 +20,9 @@ Sources of truth used here:
   * For probability targets: the hard-target oracle at one-hot targets, PyTorch's
     float64 cross_entropy with probability targets, closed forms, shift
     invariance and finite differences.
+  * For the KL divergence: PyTorch's float64 kl_div and its autograd, zero at
+    equal distributions, the two-class closed form, shift invariance, Gibbs'
+    inequality, zero-sum gradient rows and finite differences.
 """
 from __future__ import annotations
 
@@ -434,6 +437,86 @@ def pin_soft_nonfinite(orc):
     assert np.isnan(dz[2:]).all()
 
 
+# ---- KL divergence of a student from a teacher ("One barrier short") ----------------
+def pin_kl_torch_float64(orc):
+    """PyTorch float64 kl_div on log-softmaxes (log_target) and its autograd
+    with respect to the student logits, as an independent library case."""
+    torch = __import__("torch")
+    import torch.nn.functional as F
+    rng = np.random.default_rng(41)
+    zq = rng.standard_normal((6, 13)) * 4
+    zp = rng.standard_normal((6, 13)) * 4
+    g = rng.standard_normal(6)
+    qt = torch.tensor(zq, requires_grad=True)
+    ref = F.kl_div(F.log_softmax(qt, -1), F.log_softmax(torch.tensor(zp), -1), reduction="none",
+                   log_target=True).sum(-1)
+    (ref * torch.tensor(g)).sum().backward()
+    loss, _, _ = orc.kl_forward(zq, zp)
+    np.testing.assert_allclose(loss, ref.detach().numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(orc.kl_backward(zq, zp, g), qt.grad.numpy(), rtol=1e-11, atol=1e-14)
+
+
+def pin_kl_closed_forms(orc):
+    """Identical distributions: 0 and a zero gradient. Two classes:
+    a log(a/b) + (1-a) log((1-a)/(1-b)). Shifting either row by a constant
+    changes nothing; the loss is never negative (Gibbs)."""
+    rng = np.random.default_rng(42)
+    z = rng.standard_normal((4, 9))
+    loss, _, _ = orc.kl_forward(z, z)
+    assert np.abs(loss).max() <= 1e-15
+    assert np.abs(orc.kl_backward(z, z, 1.0)).max() == 0.0
+    for (x, y) in ((0.7, -1.2), (3.0, 0.0), (-2.0, 2.5)):
+        a = 1.0 / (1.0 + math.exp(-x))     # teacher p = softmax([x, 0])
+        b = 1.0 / (1.0 + math.exp(-y))     # student q = softmax([y, 0])
+        ref = a * math.log(a / b) + (1 - a) * math.log((1 - a) / (1 - b))
+        loss, _, _ = orc.kl_forward(np.array([[y, 0.0]]), np.array([[x, 0.0]]))
+        assert abs(loss[0] - ref) <= 1e-14 * max(1.0, ref)
+    zq = rng.integers(-256, 256, size=(5, 11)) / 64.0
+    zp = rng.integers(-256, 256, size=(5, 11)) / 64.0
+    l0, lq0, lp0 = orc.kl_forward(zq, zp)
+    l1, lq1, lp1 = orc.kl_forward(zq + 512.0, zp - 256.0)
+    np.testing.assert_allclose(l1, l0, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(lq1 - lq0, 512.0, rtol=1e-15)
+    np.testing.assert_allclose(lp1 - lp0, -256.0, rtol=1e-15)
+    assert (l0 >= 0).all()
+
+
+def pin_kl_grad_and_finite_differences(orc):
+    """Gradient rows sum to 0; central differences of sum_i g_i loss_i with
+    respect to the student logits."""
+    rng = np.random.default_rng(43)
+    zq = rng.standard_normal((3, 7)) * 2
+    zp = rng.standard_normal((3, 7)) * 2
+    g = rng.standard_normal(3)
+    d = orc.kl_backward(zq, zp, g)
+    assert np.abs(d.sum(1)).max() <= 1e-15
+    h = 1e-6
+    fd = np.zeros_like(zq)
+    for idx in np.ndindex(zq.shape):
+        a = zq.copy(); a[idx] += h
+        b = zq.copy(); b[idx] -= h
+        fd[idx] = (orc.kl_forward(a, zp)[0] @ g - orc.kl_forward(b, zp)[0] @ g) / (2 * h)
+    np.testing.assert_allclose(d, fd, rtol=0, atol=1e-8)
+
+
+def pin_kl_nonfinite(orc):
+    """Teacher -inf (p_j = 0) adds nothing, even over a student -inf; a
+    student -inf under teacher mass is +inf; NaN and all -inf rows give NaN."""
+    zq = np.array([[1.0, -np.inf, 0.5], [1.0, -np.inf, 0.5], [1.0, np.nan, 0.5], [0.0, 1.0, 2.0]])
+    zp = np.array([[0.5, -np.inf, 1.0], [0.5, 0.0, 1.0], [0.2, 0.3, 0.4], [-np.inf] * 3])
+    loss, lq, lp = orc.kl_forward(zq, zp)
+    lp0 = math.log(math.exp(0.5) + math.e)
+    lq0 = math.log(math.e + math.exp(0.5))
+    ref0 = (math.exp(0.5 - lp0) * ((0.5 - lp0) - (1.0 - lq0)) +
+            math.exp(1.0 - lp0) * ((1.0 - lp0) - (0.5 - lq0)))
+    assert abs(loss[0] - ref0) <= 1e-15
+    assert loss[1] == math.inf
+    assert math.isnan(loss[2]) and math.isnan(lq[2])
+    assert math.isnan(loss[3]) and lp[3] == -math.inf
+    d = orc.kl_backward(zq, zp, 1.0)
+    assert np.isfinite(d[:2]).all() and np.isnan(d[2:]).all()
+
+
 # Ordered: cheap first. The planted-mistake test runs every entry.
 BATTERY = [
     pin_pr4188_printed_values,
@@ -456,4 +539,8 @@ BATTERY = [
     pin_soft_nonfinite,
     pin_soft_torch_float64,
     pin_soft_finite_differences,
+    pin_kl_closed_forms,
+    pin_kl_nonfinite,
+    pin_kl_torch_float64,
+    pin_kl_grad_and_finite_differences,
 ]

@@ -80,6 +80,12 @@ MUTANTS = [
     ("soft grad drops g", "d[j] = g[i] * (p * T - tj);", "d[j] = (p * T - tj);"),
     ("soft grad unsmoothed target", "eps / (double)V;\n            d[j]", "0.0;\n            d[j]"),
     ("soft grad unnormalised", "const double p = exp(zr[j] - m) / s;", "const double p = exp(zr[j] - m);"),
+    ("kl uses student lse for teacher", "const double lp = p[j] - lse_p[i];", "const double lp = p[j] - lse_q[i];"),
+    ("kl sign of student term", "l += pj * (lp - (q[j] - lse_q[i]));", "l += pj * (lp + (q[j] - lse_q[i]));"),
+    ("kl weights by student", "const double pj = exp(lp);", "const double pj = exp(q[j] - lse_q[i]);"),
+    ("kl grad sign", "d[j] = g[i] * (exp(q[j] - lq) - exp(p[j] - lp));", "d[j] = g[i] * (exp(p[j] - lp) - exp(q[j] - lq));"),
+    ("kl grad drops g", "d[j] = g[i] * (exp(q[j] - lq) - exp(p[j] - lp));", "d[j] = (exp(q[j] - lq) - exp(p[j] - lp));"),
+    ("kl zero-mass terms kept", "if (pj != 0.0) l += ", "l += "),
 ]
 
 
