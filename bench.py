@@ -499,6 +499,109 @@ def bench_soft(args, rk):
     return out, None
 
 
+# -- KL divergence of a student from a teacher -------------------------------------------------
+KL_DESC = ("512 x 151,936 fp32 student and teacher logits, both ~N(0, 16) "
+           "(the shape and draw of the fused KL check in \"One barrier short\"); forward + backward")
+
+
+def kl_inputs(seed: int, N: int = 512, V: int = 151936):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((N, V), dtype=np.float32) * 4,
+            rng.standard_normal((N, V), dtype=np.float32) * 4)
+
+
+def bench_kl(args, rk):
+    import torch
+    import softmax_cross_entropy_lse_b200 as ce
+    world = rk.world
+    q, p = kl_inputs(rk.rank)
+    if args.rows:
+        q, p = q[:args.rows], p[:args.rows]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q_h, p_h = torch.from_numpy(q), torch.from_numpy(p)
+    q_d, p_d = q_h.to(dev), p_h.to(dev)
+    N, V = q_d.shape
+    g = torch.full((1,), 1.0 / N, dtype=torch.float32, device=dev)
+    dq = torch.empty_like(q_d)
+    stream = torch.cuda.current_stream()
+    fwd_bytes = 2 * N * V * 4 + 20 * N
+    bwd_bytes = 3 * N * V * 4 + 20 * N
+    step_bytes = fwd_bytes + bwd_bytes
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        r = ce.kl_forward(q_d, p_d)
+        if ev is not None:
+            ev[1].record(stream)
+        ce.kl_backward(g, q_d, p_d, r, dstudent=dq)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clk:
+        sharding.barrier(rk)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        sharding.barrier(rk)
+    ms = sharding.max_over_ranks(rk, t0.elapsed_time(t1))
+    fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    q_pin, p_pin = q_h.pin_memory(), p_h.pin_memory()
+    loss_h = torch.empty(N, dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        q_d.copy_(q_pin, non_blocking=True)
+        p_d.copy_(p_pin, non_blocking=True)
+        r = ce.kl_forward(q_d, p_d)
+        ce.kl_backward(g, q_d, p_d, r, dstudent=dq)
+        loss_h.copy_(r.loss, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    sharding.barrier(rk)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(3):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sharding.max_over_ranks(rk, a.elapsed_time(b)) / 3
+    peak_hbm, _, _, peak_src = load_peaks()
+    dom, dom_ms, dom_bytes = ("backward", bwd_ms, bwd_bytes) if bwd_ms >= fwd_ms else \
+        ("forward", fwd_ms, fwd_bytes)
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    out = {
+        "metric": METRIC, "value": round(world * step_bytes * args.steps / (ms * 1e-3) / 1e9, 2),
+        "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "fwd_GBs": round(fwd_bytes / (fwd_ms * 1e-3) / 1e9, 2),
+        "bwd_GBs": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9, 2),
+        "config": {"workload": f"kl: {KL_DESC}", "rows": N, "classes": V,
+                   "bytes_per_step": step_bytes, "l2": "inputs larger than L2",
+                   "parallelism": f"rows sharded over {world} rank(s), no data-path collective"},
+        "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": 2 * N * V * 4, "d2h_bytes_per_step": 4 * N},
+        "gpu_launches": 2 * args.steps,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 2), "peak": peak_hbm,
+                     "unit": "GB/s", "frac": round(achieved / peak_hbm, 4), "traffic": None,
+                     "peak_source": peak_src, "algorithmic_bytes_per_launch": dom_bytes},
+    }
+    clocks = clk.summary()
+    if clocks:
+        out["clocks"] = clocks
+    return out, None
+
+
 # -- fused-linear workload -------------------------------------------------------------------
 def bench_linear(args, rk):
     import torch
@@ -699,6 +802,39 @@ class OracleSoft(OracleRows):
             done += n
 
 
+class OracleKl(OracleRows):
+    """The float64 oracle for the KL divergence (forward + backward)."""
+
+    def __init__(self):
+        import oracle
+        self.orc = oracle.get()
+        self.q32, self.p32 = kl_inputs(0)
+        self.N, self.V = self.q32.shape
+        self.bytes_per_row = 5 * self.V * 4 + 40
+        self.cursor = 0
+
+    def run(self, rows: int) -> None:
+        done = 0
+        chunk = max(1, int(5e7 // self.V))
+        while done < rows:
+            lo = self.cursor % self.N
+            n = min(chunk, rows - done, self.N - lo)
+            q = self.q32[lo:lo + n].astype(np.float64)
+            p = self.p32[lo:lo + n].astype(np.float64)
+            self.orc.kl_forward(q, p)
+            self.orc.kl_backward(q, p, 1.0)
+            self.cursor += n
+            done += n
+
+
+def _oracle_for(workload, host=None):
+    if workload == "soft":
+        return OracleSoft()
+    if workload == "kl":
+        return OracleKl()
+    return OracleRows(workload, host)
+
+
 def oracle_baseline(workload, seconds: float, host=None):
     """(value, unit, cores, sample) of the oracle timed for about `seconds`."""
     if workload == "c5":
@@ -709,7 +845,7 @@ def oracle_baseline(workload, seconds: float, host=None):
         dt = time.perf_counter() - t
         return (rows * o.flop_per_row / dt / 1e12, "TFLOP/s", o.orc.num_threads(),
                 f"{rows} of 8192 rows of c5 (loss, lse and dH rows), {dt:.1f} s")
-    o = OracleSoft() if workload == "soft" else OracleRows(workload, host)
+    o = _oracle_for(workload, host)
     rows = min(o.rows_for(seconds), 50 * o.N)
     t = time.perf_counter()
     o.run(rows)
@@ -727,7 +863,7 @@ def run_reference(args):
         o = OracleLinear()
         unit, per_row = "TFLOP/s", o.flop_per_row / 1e12
     else:
-        o = OracleSoft() if args.workload == "soft" else OracleRows(args.workload)
+        o = _oracle_for(args.workload)
         unit, per_row = "GB/s", o.bytes_per_row / 1e9
     # each step a bounded sample, so the whole run stays within about two minutes
     step_s = min(2.0, 120.0 / (args.steps + args.warmup))
@@ -761,7 +897,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="c2", choices=sorted(ROW_WORKLOADS) + ["c5", "soft"])
+    ap.add_argument("--workload", default="c2", choices=sorted(ROW_WORKLOADS) + ["c5", "soft", "kl"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rows", type=int, default=0,
@@ -782,6 +918,8 @@ def main():
         out, host = bench_linear(args, rk)
     elif args.workload == "soft":
         out, host = bench_soft(args, rk)
+    elif args.workload == "kl":
+        out, host = bench_kl(args, rk)
     else:
         out, host = bench_rows(args, rk)
     if rk.rank == 0 and rk.world == 1 and not args.no_cpu_baseline:

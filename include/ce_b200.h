@@ -207,6 +207,39 @@ ce_status ce_soft_backward(const float* grad_out, int64_t grad_stride,
                            void* cuda_stream);
 
 /* ------------------------------------------------------------------------ *
+ * KL divergence of a student distribution from a teacher's, fused. Source:
+ * Suryavanshi, "One barrier short" (the fused KL loss of mlx-lm, forward and
+ * backward in one pass over both rows, an online log-sum-exp for each). With
+ * teacher logits zp and student logits zq of a row, p = softmax(zp) and
+ * q = softmax(zq):
+ *     loss_i = sum_j p_ij (log p_ij - log q_ij),   dzq_ij = g_i (q_ij - p_ij).
+ * Only the student gets a gradient (the teacher is a fixed target). A class
+ * with p_ij = 0 adds nothing, even where zq_ij is -inf too; a student -inf
+ * under teacher mass gives +inf. NaN in either row, or a row of either that
+ * is all -inf, gives a NaN loss and a NaN gradient row. Both inputs have
+ * dtype dt (f32, bf16, f16), N x V through their own layouts. The result
+ * depends on the inputs alone: repeated calls give the same bytes (the
+ * cross-lane exchange reuses no scratch, so the race "One barrier short"
+ * describes cannot occur).
+ * ------------------------------------------------------------------------ */
+
+/* Forward: loss, the student's and the teacher's lse (each with its lo
+ * part, nullable, as in ce_forward). N floats each. No workspace. */
+ce_status ce_kl_forward(const void* student, const void* teacher, ce_dtype dt, ce_layout ls,
+                        ce_layout lt, int64_t N, int64_t V, float* loss, float* lse_student,
+                        float* lse_student_lo, float* lse_teacher, float* lse_teacher_lo,
+                        void* cuda_stream);
+
+/* Backward: dstudent (dtype ddt: dt or f32; may be the student logits
+ * themselves, same pointer, dtype and layout) from the saved lse pairs.
+ * grad_out and grad_stride as for ce_backward. */
+ce_status ce_kl_backward(const float* grad_out, int64_t grad_stride, const void* student,
+                         const void* teacher, ce_dtype dt, ce_layout ls, ce_layout lt, int64_t N,
+                         int64_t V, const float* lse_student, const float* lse_student_lo,
+                         const float* lse_teacher, const float* lse_teacher_lo, void* dstudent,
+                         ce_dtype ddt, ce_layout dl, void* cuda_stream);
+
+/* ------------------------------------------------------------------------ *
  * Fused-linear cross-entropy: logits Z = H W^T are never stored.
  * Source: Ineshin, "A fused linear cross-entropy forward kernel for Apple
  * GPUs", section 1 (Z = H W^T streamed over vocabulary tiles into the running

@@ -26,7 +26,7 @@ STATUS = {0: "CE_OK", 1: "CE_EINVAL", 2: "CE_EALIAS", 3: "CE_EWORKSPACE", 4: "CE
 EXPORTED = ["ce_workspace_size", "ce_forward", "ce_backward", "linear_ce_workspace_size",
             "linear_ce_forward", "linear_ce_backward_workspace_size", "linear_ce_backward",
             "ce_get_error", "ce_status_string", "ce_forward_noalloc", "ce_forward_backward",
-            "ce_soft_forward", "ce_soft_backward"]
+            "ce_soft_forward", "ce_soft_backward", "ce_kl_forward", "ce_kl_backward"]
 NOALLOC_SCRATCH_BYTES = 64 << 10
 
 
@@ -85,6 +85,12 @@ def lib() -> ctypes.CDLL:
         L.ce_soft_backward.argtypes = [vp, i64, vp, ctypes.c_int, ce_layout, i64, i64, vp, ctypes.c_int,
                                        ce_layout, vp, vp, vp, f32, vp, ctypes.c_int, ce_layout, vp]
         L.ce_soft_backward.restype = ctypes.c_int
+        L.ce_kl_forward.argtypes = [vp, vp, ctypes.c_int, ce_layout, ce_layout, i64, i64, vp, vp, vp, vp,
+                                    vp, vp]
+        L.ce_kl_forward.restype = ctypes.c_int
+        L.ce_kl_backward.argtypes = [vp, i64, vp, vp, ctypes.c_int, ce_layout, ce_layout, i64, i64, vp,
+                                     vp, vp, vp, vp, ctypes.c_int, ce_layout, vp]
+        L.ce_kl_backward.restype = ctypes.c_int
         L.ce_get_error.argtypes = [vp]
         L.ce_get_error.restype = ctypes.c_int
         L.ce_status_string.argtypes = [ctypes.c_int]
@@ -349,6 +355,61 @@ def ce_soft_backward(grad_out, logits, target_probs, lse, lse_lo=None, target_su
                                     _ptr(dlogits), _dtype_code(dlogits), dl, _stream(stream))
     _check(st, "ce_soft_backward")
     return dlogits
+
+
+class KlResult(NamedTuple):
+    loss: object
+    lse_student: object
+    lse_student_lo: object
+    lse_teacher: object
+    lse_teacher_lo: object
+
+
+def _same_rows(a, b, what):
+    Na, la = row_layout(a, True)
+    Nb, lb = row_layout(b, True)
+    if Na != Nb or a.shape[-1] != b.shape[-1]:
+        raise ValueError(f"{what} must have the shape of the student logits")
+    return Na, la, lb
+
+
+def kl_forward(student, teacher, *, stream=None) -> KlResult:
+    """KL(softmax(teacher) || softmax(student)) per row, with both lse pairs.
+    student and teacher: same shape and dtype, any strides."""
+    torch = _torch()
+    _require_cuda(student, teacher)
+    if teacher.dtype != student.dtype:
+        raise TypeError("student and teacher logits must share a dtype")
+    N, ls, lt = _same_rows(student, teacher, "teacher logits")
+    V = student.shape[-1]
+    dev = student.device
+    outs = [torch.empty(N, dtype=torch.float32, device=dev) for _ in range(5)]
+    with torch.cuda.device(dev):
+        st = lib().ce_kl_forward(_ptr(student), _ptr(teacher), _dtype_code(student), ls, lt, N, V,
+                                 *[_ptr(o) for o in outs], _stream(stream))
+    _check(st, "ce_kl_forward")
+    return KlResult(*outs)
+
+
+def kl_backward(grad_out, student, teacher, r: KlResult, *, dstudent=None, out_dtype=None, stream=None):
+    """g (softmax(student) - softmax(teacher)) from kl_forward's lse pairs."""
+    torch = _torch()
+    _require_cuda(grad_out, student, teacher, dstudent)
+    N, ls, lt = _same_rows(student, teacher, "teacher logits")
+    V = student.shape[-1]
+    grad_out, g_stride = _grad_view(torch, grad_out, N)
+    if dstudent is None:
+        dstudent = torch.empty(student.shape, dtype=out_dtype or student.dtype, device=student.device)
+    Nd, dl = row_layout(dstudent, True)
+    if Nd != N or dstudent.shape[-1] != V:
+        raise ValueError("dstudent must have the shape of the student logits")
+    with torch.cuda.device(student.device):
+        st = lib().ce_kl_backward(_ptr(grad_out), g_stride, _ptr(student), _ptr(teacher),
+                                  _dtype_code(student), ls, lt, N, V, _ptr(r.lse_student),
+                                  _ptr(r.lse_student_lo), _ptr(r.lse_teacher), _ptr(r.lse_teacher_lo),
+                                  _ptr(dstudent), _dtype_code(dstudent), dl, _stream(stream))
+    _check(st, "ce_kl_backward")
+    return dstudent
 
 
 def ce_forward_backward(logits, targets, grad_out, label_smoothing: float = 0.0,

@@ -475,6 +475,98 @@ ce_status ce_soft_backward(const float* grad_out, int64_t grad_stride, const voi
     return e == cudaSuccess ? CE_OK : CE_ECUDA;
 }
 
+// ---- KL divergence of a student from a teacher -------------------------------------
+ce_status ce_kl_forward(const void* student, const void* teacher, ce_dtype dt, ce_layout ls,
+                        ce_layout lt, int64_t N, int64_t V, float* loss, float* lse_student,
+                        float* lse_student_lo, float* lse_teacher, float* lse_teacher_lo,
+                        void* cuda_stream) {
+    if (N < 0 || V < 1 || V > INT32_MAX) return CE_EINVAL;
+    if (dt != CE_F32 && dt != CE_BF16 && dt != CE_F16) return CE_EINVAL;
+    if (N == 0) return CE_OK;
+    if (!student || !teacher || !loss || !lse_student || !lse_teacher) return CE_EINVAL;
+    if (!layout_ok(ls) || !layout_ok(lt)) return CE_EINVAL;
+    const int esz = elem_size(dt);
+    const Layout Q = to_layout(ls), P = to_layout(lt);
+    const Extent eq = layout_extent(student, Q, N, V, esz);
+    const Extent ep = layout_extent(teacher, P, N, V, esz);
+    Extent outs[5];
+    int nout = 0;
+    outs[nout++] = flat_extent(loss, N, 4);
+    outs[nout++] = flat_extent(lse_student, N, 4);
+    outs[nout++] = flat_extent(lse_teacher, N, 4);
+    if (lse_student_lo) outs[nout++] = flat_extent(lse_student_lo, N, 4);
+    if (lse_teacher_lo) outs[nout++] = flat_extent(lse_teacher_lo, N, 4);
+    for (int i = 0; i < nout; ++i) {
+        if (overlap(outs[i], eq) || overlap(outs[i], ep)) return CE_EALIAS;
+        for (int j = 0; j < i; ++j)
+            if (overlap(outs[i], outs[j])) return CE_EALIAS;
+    }
+    const bool vec_ok = vectorizable(student, Q, N, esz) && vectorizable(teacher, P, N, esz);
+    KlPlan p = plan_soft(N, V, esz, esz, vec_ok, device_sms(0));
+    KlArgs a{};
+    a.zq = student;
+    a.zp = teacher;
+    a.N = N;
+    a.V = V;
+    a.loss = loss;
+    a.lse_q = lse_student;
+    a.lse_q_lo = lse_student_lo;
+    a.lse_p = lse_teacher;
+    a.lse_p_lo = lse_teacher_lo;
+    a.lq = Q;
+    a.lp = P;
+    cudaError_t e = launch_kl_forward(p, a, (int)dt, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? CE_OK : CE_ECUDA;
+}
+
+ce_status ce_kl_backward(const float* grad_out, int64_t grad_stride, const void* student,
+                         const void* teacher, ce_dtype dt, ce_layout ls, ce_layout lt, int64_t N,
+                         int64_t V, const float* lse_student, const float* lse_student_lo,
+                         const float* lse_teacher, const float* lse_teacher_lo, void* dstudent,
+                         ce_dtype ddt, ce_layout dl, void* cuda_stream) {
+    if (N < 0 || V < 1 || V > INT32_MAX) return CE_EINVAL;
+    if (dt != CE_F32 && dt != CE_BF16 && dt != CE_F16) return CE_EINVAL;
+    if (ddt != CE_F32 && ddt != dt) return CE_ENOTSUP;
+    if (N == 0) return CE_OK;
+    if (!grad_out || !student || !teacher || !lse_student || !lse_teacher || !dstudent) return CE_EINVAL;
+    if (!layout_ok(ls) || !layout_ok(lt) || !layout_ok(dl)) return CE_EINVAL;
+    const int esz = elem_size(dt), dsz = elem_size(ddt);
+    const Layout Q = to_layout(ls), P = to_layout(lt), D = to_layout(dl);
+    const Extent eq = layout_extent(student, Q, N, V, esz);
+    const Extent ep = layout_extent(teacher, P, N, V, esz);
+    const Extent ed = layout_extent(dstudent, D, N, V, dsz);
+    const Extent eg = grad_stride == 0 ? flat_extent(grad_out, 1, 4)
+                                       : layout_extent(grad_out, Layout{N, 0, grad_stride, 0}, N, 1, 4);
+    const bool in_place = dstudent == student && ddt == dt && Q.inner == D.inner &&
+                          Q.s_outer == D.s_outer && Q.s_inner == D.s_inner && Q.s_col == D.s_col;
+    if (!in_place && overlap(ed, eq)) return CE_EALIAS;
+    if (overlap(ed, ep) || overlap(ed, eg) || overlap(ed, flat_extent(lse_student, N, 4)) ||
+        overlap(ed, flat_extent(lse_teacher, N, 4)))
+        return CE_EALIAS;
+    if (lse_student_lo && overlap(ed, flat_extent(lse_student_lo, N, 4))) return CE_EALIAS;
+    if (lse_teacher_lo && overlap(ed, flat_extent(lse_teacher_lo, N, 4))) return CE_EALIAS;
+    const bool vec_ok = vectorizable(student, Q, N, esz) && vectorizable(teacher, P, N, esz) &&
+                        vectorizable(dstudent, D, N, dsz);
+    KlPlan p = plan_soft(N, V, esz, esz, vec_ok, device_sms(0));
+    KlArgs a{};
+    a.zq = student;
+    a.zp = teacher;
+    a.N = N;
+    a.V = V;
+    a.lse_q = const_cast<float*>(lse_student);
+    a.lse_q_lo = const_cast<float*>(lse_student_lo);
+    a.lse_p = const_cast<float*>(lse_teacher);
+    a.lse_p_lo = const_cast<float*>(lse_teacher_lo);
+    a.g = grad_out;
+    a.g_stride = grad_stride;
+    a.dz = dstudent;
+    a.lq = Q;
+    a.lp = P;
+    a.ld = D;
+    cudaError_t e = launch_kl_backward(p, a, (int)dt, (int)ddt, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? CE_OK : CE_ECUDA;
+}
+
 ce_status ce_forward_backward(const void* logits, ce_dtype dt, ce_layout lg, int64_t N, int64_t V,
                               const void* targets, ce_index_dtype tdt, ce_layout tg,
                               float label_smoothing, int64_t ignore_index, const float* grad_out,

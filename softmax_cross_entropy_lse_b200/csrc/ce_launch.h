@@ -143,4 +143,25 @@ cudaError_t launch_soft_forward(const SoftPlan& p, const SoftArgs& a, int dz_t, 
 cudaError_t launch_soft_backward(const SoftPlan& p, const SoftArgs& a, int dz_t, int dt_t, int do_t,
                                  cudaStream_t s);
 
+// ---- KL divergence of a student (q) from a teacher (p) ----------------------
+struct KlArgs {
+    const void* zq;   // student logits
+    const void* zp;   // teacher logits
+    int64_t N, V;
+    float* loss;
+    float* lse_q;
+    float* lse_q_lo;
+    float* lse_p;
+    float* lse_p_lo;
+    const float* g;   // backward
+    int64_t g_stride;
+    void* dz;
+    Layout lq, lp, ld;
+};
+
+using KlPlan = SoftPlan;
+
+cudaError_t launch_kl_forward(const KlPlan& p, const KlArgs& a, int dt, cudaStream_t s);
+cudaError_t launch_kl_backward(const KlPlan& p, const KlArgs& a, int dt, int ddt, cudaStream_t s);
+
 }  // namespace ceb

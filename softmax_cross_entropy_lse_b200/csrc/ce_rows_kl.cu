@@ -1,0 +1,282 @@
+// KL divergence of a student distribution from a teacher's, fused.
+//
+// Suryavanshi, "One barrier short", describes the fused KL loss of mlx-lm:
+// for teacher logits zp and student logits zq of a row, p = softmax(zp) and
+// q = softmax(zq),
+//     loss = sum_j p_j (log p_j - log q_j),   dzq_j = g (q_j - p_j),
+// computed in one pass with an online log-sum-exp per distribution. With
+// (mq, sq) and (mp, sp) the running max and scaled sum of each, and
+//     W = sum_j exp(zp_j - mp) (zp_j - zq_j),
+// rescaled by exp(mp - mp') together with sp whenever mp grows to mp',
+//     loss = W / sp - (lse_p - lse_q).
+// A class with p_j = 0 adds nothing to W, even where zq_j is -inf too
+// (0 log 0 = 0). The backward recomputes q_j and p_j from the two saved
+// (lse, lse_lo) pairs.
+//
+// G lanes share a row (a whole warp, looping, for long rows), 32 / G rows
+// per warp, grid-stride over rows; both rows stay in flight as raw 16-byte
+// words. The cross-lane merge takes each maximum first, so the exchange has
+// no slot to reuse (the race that "One barrier short" is about cannot occur).
+#include "ce_device.cuh"
+#include "ce_launch.h"
+
+namespace ceb {
+
+struct KlState {
+    float mq, sq, mp, sp, w;
+};
+
+__device__ __forceinline__ void kl_rescale(KlState& st, float mq, float mp) {
+    if (st.mq != mq) {
+        st.sq *= ex2((st.mq - mq) * kLog2e);
+        st.mq = mq;
+    }
+    if (st.mp != mp) {
+        const float f = ex2((st.mp - mp) * kLog2e);
+        st.sp *= f;
+        st.w *= f;
+        st.mp = mp;
+    }
+}
+
+template <int n>
+__device__ __forceinline__ void kl_fold(KlState& st, const float (&zq)[n], const float (&zp)[n]) {
+    float cq = zq[0], cp = zp[0];
+#pragma unroll
+    for (int i = 1; i < n; ++i) {
+        cq = fmaxf(cq, zq[i]);
+        cp = fmaxf(cp, zp[i]);
+    }
+    kl_rescale(st, fmaxf(st.mq, cq), fmaxf(st.mp, cp));
+    const float msq = st.mq == -INFINITY ? 0.f : st.mq;
+    const float msp = st.mp == -INFINITY ? 0.f : st.mp;
+    float sq = 0.f, sp = 0.f, w = 0.f;
+#pragma unroll
+    for (int i = 0; i < n; ++i) {
+        sq += ex2((zq[i] - msq) * kLog2e);
+        const float ep = ex2((zp[i] - msp) * kLog2e);
+        sp += ep;
+        if (ep != 0.f) w = fmaf(ep, zp[i] - zq[i], w);
+    }
+    st.sq += sq;
+    st.sp += sp;
+    st.w += w;
+}
+
+template <int G>
+__device__ __forceinline__ void kl_group_reduce(KlState& st) {
+    if constexpr (G > 1) {
+        float Mq = st.mq, Mp = st.mp;
+#pragma unroll
+        for (int off = G / 2; off >= 1; off >>= 1) {
+            Mq = fmaxf(Mq, __shfl_xor_sync(0xffffffffu, Mq, off));
+            Mp = fmaxf(Mp, __shfl_xor_sync(0xffffffffu, Mp, off));
+        }
+        kl_rescale(st, Mq, Mp);
+#pragma unroll
+        for (int off = G / 2; off >= 1; off >>= 1) {
+            st.sq += __shfl_xor_sync(0xffffffffu, st.sq, off);
+            st.sp += __shfl_xor_sync(0xffffffffu, st.sp, off);
+            st.w += __shfl_xor_sync(0xffffffffu, st.w, off);
+        }
+    }
+}
+
+template <typename T, int VEC, int G, int U, int MINB>
+__global__ void __launch_bounds__(256, MINB) k_kl_fwd(KlArgs a) {
+    const T* __restrict__ zs = reinterpret_cast<const T*>(a.zq);
+    const T* __restrict__ zt = reinterpret_cast<const T*>(a.zp);
+    const int lane = threadIdx.x & 31;
+    const int gl = lane & (G - 1);
+    constexpr int kRowsPerStep = 32 / G;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t nvec = a.V / VEC;
+    const int tail = (int)(a.V - nvec * VEC);
+
+    for (int64_t base = warp * kRowsPerStep; base < a.N; base += nwarps * kRowsPerStep) {
+        const int64_t r = base + lane / G;
+        const bool active = r < a.N;
+        KlState st{-INFINITY, 0.f, -INFINITY, 0.f, 0.f};
+        const T* qr = zs;
+        const T* pr = zt;
+        if (active) {
+            qr = zs + row_offset(a.lq, r, a.N);
+            pr = zt + row_offset(a.lp, r, a.N);
+        }
+        for (int64_t vb = 0; vb < nvec; vb += (int64_t)G * U) {
+            Raw<T, VEC> rq[U], rp[U];
+            bool ok[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t vi = vb + u * G + gl;
+                ok[u] = active && vi < nvec;
+                if (ok[u]) {
+                    load_raw<T, VEC>(qr, vi * VEC, a.lq.s_col, rq[u]);
+                    load_raw<T, VEC>(pr, vi * VEC, a.lp.s_col, rp[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (!ok[u]) continue;
+                float q[VEC], p[VEC];
+                unpack_raw<T, VEC>(rq[u], q);
+                unpack_raw<T, VEC>(rp[u], p);
+                kl_fold<VEC>(st, q, p);
+            }
+        }
+        if (active) {
+            for (int c = gl; c < tail; c += G) {
+                const int64_t col = nvec * VEC + c;
+                const float q[1] = {to_f32(qr[col * a.lq.s_col])};
+                const float p[1] = {to_f32(pr[col * a.lp.s_col])};
+                kl_fold<1>(st, q, p);
+            }
+        }
+        kl_group_reduce<G>(st);
+        if (active && gl == 0) {
+            OnlineState oq = empty_state(), op = empty_state();
+            oq.m = st.mq;
+            oq.s = st.sq;
+            op.m = st.mp;
+            op.s = st.sp;
+            float Lq, hq, lq, Lp, hp, lp;
+            lse_pair(oq, Lq, hq, lq);
+            lse_pair(op, Lp, hp, lp);
+            a.lse_q[r] = hq;
+            a.lse_p[r] = hp;
+            if (a.lse_q_lo) a.lse_q_lo[r] = lq;
+            if (a.lse_p_lo) a.lse_p_lo[r] = lp;
+            float loss = __int_as_float(0x7fc00000);
+            if (isfinite(hq) && isfinite(hp)) loss = st.w / st.sp - (st.mp - st.mq) - (Lp - Lq);
+            a.loss[r] = loss;
+        }
+    }
+}
+
+template <typename T, typename TO, int VEC, int G, int U, int MINB>
+__global__ void __launch_bounds__(256, MINB) k_kl_bwd(KlArgs a) {
+    const T* zs = reinterpret_cast<const T*>(a.zq);
+    const T* __restrict__ zt = reinterpret_cast<const T*>(a.zp);
+    TO* dz = reinterpret_cast<TO*>(a.dz);
+    const int lane = threadIdx.x & 31;
+    const int gl = lane & (G - 1);
+    constexpr int kRowsPerStep = 32 / G;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t nvec = a.V / VEC;
+    const int tail = (int)(a.V - nvec * VEC);
+
+    for (int64_t base = warp * kRowsPerStep; base < a.N; base += nwarps * kRowsPerStep) {
+        const int64_t r = base + lane / G;
+        if (r >= a.N) continue;
+        const T* qr = zs + row_offset(a.lq, r, a.N);
+        const T* pr = zt + row_offset(a.lp, r, a.N);
+        TO* dr = dz + row_offset(a.ld, r, a.N);
+        const float g = a.g[r * a.g_stride];
+        const float hq = a.lse_q[r], hp = a.lse_p[r];
+        const float cq = (a.lse_q_lo ? a.lse_q_lo[r] : 0.f) * kLog2e;
+        const float cp = (a.lse_p_lo ? a.lse_p_lo[r] : 0.f) * kLog2e;
+        // a row whose lse is not finite has no distribution: NaN gradient
+        const bool bad = !isfinite(hq) || !isfinite(hp);
+        for (int64_t vb = gl; vb < nvec; vb += (int64_t)G * U) {
+            Raw<T, VEC> rq[U], rp[U];
+            bool ok[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t vi = vb + (int64_t)u * G;
+                ok[u] = vi < nvec;
+                if (ok[u]) {
+                    load_raw<T, VEC>(qr, vi * VEC, a.lq.s_col, rq[u]);
+                    load_raw<T, VEC>(pr, vi * VEC, a.lp.s_col, rp[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (!ok[u]) continue;
+                float q[VEC], p[VEC], o[VEC];
+                unpack_raw<T, VEC>(rq[u], q);
+                unpack_raw<T, VEC>(rp[u], p);
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    const float qe = ex2(fmaf(q[e] - hq, kLog2e, -cq));
+                    const float pe = ex2(fmaf(p[e] - hp, kLog2e, -cp));
+                    o[e] = bad ? __int_as_float(0x7fc00000) : g * (qe - pe);
+                }
+                store_vec<TO, VEC>(dr, (vb + (int64_t)u * G) * VEC, a.ld.s_col, o);
+            }
+        }
+        for (int c = gl; c < tail; c += G) {
+            const int64_t col = nvec * VEC + c;
+            const float qe = ex2(fmaf(to_f32(qr[col * a.lq.s_col]) - hq, kLog2e, -cq));
+            const float pe = ex2(fmaf(to_f32(pr[col * a.lp.s_col]) - hp, kLog2e, -cp));
+            cvt_store1(dr + col * a.ld.s_col, bad ? __int_as_float(0x7fc00000) : g * (qe - pe));
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Four vectors of each row in flight per lane (eight on the scalar path) at
+// three blocks per SM: two rows' words take the registers of four blocks'
+// worth. The planner's lane grouping uses the same U.
+template <int VEC, bool BWD = false> struct KlShape {
+    static constexpr int U = VEC == 1 ? 8 : 4;
+    static constexpr int MINB = VEC == 1 ? 2 : 3;
+};
+
+template <typename T, int VEC>
+static cudaError_t kl_fwd_v(const KlPlan& p, const KlArgs& a, cudaStream_t s) {
+    constexpr int U = KlShape<VEC>::U, MB = KlShape<VEC>::MINB;
+#define CEB_KL(GG)                                                          \
+    if (p.G == GG) {                                                        \
+        k_kl_fwd<T, VEC, GG, U, MB><<<p.grid, 256, 0, s>>>(a);              \
+        return cudaGetLastError();                                          \
+    }
+    CEB_KL(1) CEB_KL(2) CEB_KL(4) CEB_KL(8) CEB_KL(16) CEB_KL(32)
+#undef CEB_KL
+    return cudaErrorInvalidValue;
+}
+
+template <typename T, typename TO, int VEC>
+static cudaError_t kl_bwd_v(const KlPlan& p, const KlArgs& a, cudaStream_t s) {
+    constexpr int U = KlShape<VEC, true>::U, MB = KlShape<VEC, true>::MINB;
+#define CEB_KL(GG)                                                          \
+    if (p.G == GG) {                                                        \
+        k_kl_bwd<T, TO, VEC, GG, U, MB><<<p.grid, 256, 0, s>>>(a);          \
+        return cudaGetLastError();                                          \
+    }
+    CEB_KL(1) CEB_KL(2) CEB_KL(4) CEB_KL(8) CEB_KL(16) CEB_KL(32)
+#undef CEB_KL
+    return cudaErrorInvalidValue;
+}
+
+template <typename T>
+static cudaError_t kl_fwd_t(const KlPlan& p, const KlArgs& a, cudaStream_t s) {
+    if (p.vec == 1) return kl_fwd_v<T, 1>(p, a, s);
+    return kl_fwd_v<T, ElemTraits<T>::kVec>(p, a, s);
+}
+
+template <typename T, typename TO>
+static cudaError_t kl_bwd_t(const KlPlan& p, const KlArgs& a, cudaStream_t s) {
+    if (p.vec == 1) return kl_bwd_v<T, TO, 1>(p, a, s);
+    return kl_bwd_v<T, TO, ElemTraits<T>::kVec>(p, a, s);
+}
+
+cudaError_t launch_kl_forward(const KlPlan& p, const KlArgs& a, int dt, cudaStream_t s) {
+    switch (dt) {
+        case 0: return kl_fwd_t<float>(p, a, s);
+        case 1: return kl_fwd_t<__nv_bfloat16>(p, a, s);
+        case 2: return kl_fwd_t<__half>(p, a, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_kl_backward(const KlPlan& p, const KlArgs& a, int dt, int ddt, cudaStream_t s) {
+    if (dt == 0) return kl_bwd_t<float, float>(p, a, s);
+    if (dt == 1) return ddt == 0 ? kl_bwd_t<__nv_bfloat16, float>(p, a, s)
+                                 : kl_bwd_t<__nv_bfloat16, __nv_bfloat16>(p, a, s);
+    if (dt == 2) return ddt == 0 ? kl_bwd_t<__half, float>(p, a, s) : kl_bwd_t<__half, __half>(p, a, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace ceb

@@ -42,36 +42,6 @@ __device__ __forceinline__ void load_n(const T* p, int64_t col, int64_t s_col, f
     }
 }
 
-// VEC elements of T held as raw 16-byte words (VEC > 1) or one float (VEC =
-// 1) between the load and the use, so that many loads can be in flight in
-// few registers.
-template <typename T, int VEC>
-struct Raw {
-    static constexpr int W = VEC == 1 ? 1 : (int)(VEC * sizeof(T) / 16);
-    uint4 w[W];
-};
-
-template <typename T, int VEC>
-__device__ __forceinline__ void load_raw(const T* p, int64_t col, int64_t s_col, Raw<T, VEC>& r) {
-    if constexpr (VEC == 1) {
-        r.w[0].x = __float_as_uint(to_f32(p[col * s_col]));
-    } else {
-#pragma unroll
-        for (int w = 0; w < Raw<T, VEC>::W; ++w) r.w[w] = __ldcs(reinterpret_cast<const uint4*>(p + col) + w);
-    }
-}
-
-template <typename T, int VEC>
-__device__ __forceinline__ void unpack_raw(const Raw<T, VEC>& r, float (&out)[VEC]) {
-    if constexpr (VEC == 1) {
-        out[0] = __uint_as_float(r.w[0].x);
-    } else {
-        constexpr int PER = 16 / (int)sizeof(T);
-#pragma unroll
-        for (int w = 0; w < Raw<T, VEC>::W; ++w) unpack_words<T>(r.w[w], out + w * PER);
-    }
-}
-
 template <bool EPS>
 __device__ __forceinline__ void soft_rescale(SoftState& st, float mn) {
     if (st.m != mn) {

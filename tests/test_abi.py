@@ -214,3 +214,25 @@ def test_soft_targets_reject_bad_arguments_and_aliasing(L):
     assert soft_bwd(L, dz=T + 64) == 2        # gradient over the targets
     assert soft_bwd(L, dz=OUT) == 2           # gradient over lse
     assert soft_bwd(L, g=None) == 1
+
+
+def test_kl_rejects_bad_arguments_and_aliasing(L):
+    N, V = 8, 16
+
+    def fwd_kl(q=Z, p=T, dt=0, loss=OUT, lq=OUT + 4096, lp=OUT + 8192, lq_lo=None, lp_lo=None, n=N):
+        return L.ce_kl_forward(q, p, dt, lay(n, V), lay(n, V), n, V, loss, lq, lq_lo, lp, lp_lo, None)
+
+    def bwd_kl(g=OUT + 16384, dq=0x40000000, ddt=0, dt=0):
+        return L.ce_kl_backward(g, 0, Z, T, dt, lay(N, V), lay(N, V), N, V, OUT, None, OUT + 4096, None,
+                                dq, ddt, lay(N, V), None)
+
+    assert fwd_kl(dt=5) == 1
+    assert fwd_kl(p=None) == 1
+    assert fwd_kl(lp=None) == 1
+    assert fwd_kl(n=0, q=None, p=None, loss=None, lq=None, lp=None) == 0
+    assert fwd_kl(loss=T + 8) == 2          # loss over the teacher logits
+    assert fwd_kl(lp=OUT + 4096 + 16) == 2  # teacher lse over the student lse
+    assert bwd_kl(ddt=1) == 6               # bf16 gradient of f32 logits
+    assert bwd_kl(dq=T) == 2                # gradient over the teacher
+    assert bwd_kl(dq=OUT + 4096) == 2       # gradient over the teacher lse
+    assert bwd_kl(g=None) == 1
