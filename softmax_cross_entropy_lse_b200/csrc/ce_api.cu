@@ -476,6 +476,25 @@ ce_status ce_soft_backward(const float* grad_out, int64_t grad_stride, const voi
 }
 
 // ---- KL divergence of a student from a teacher -------------------------------------
+// Rows that need a whole warp (G = 32) and number fewer than the resident
+// warps of the GPU take a CTA each in the forward and (row, 1024-vector
+// chunk) units in the backward.
+static KlPlan plan_kl(int64_t N, int64_t V, int esz, bool vec_ok, int sms) {
+    KlPlan p = plan_soft(N, V, esz, esz, vec_ok, sms);
+    p.cta = 0;
+    if (p.G == 32 && N < (int64_t)sms * 24) {
+        p.cta = 1;
+        const int64_t cap = (int64_t)sms * 4;
+        p.grid = (int)(N < cap ? (N > 0 ? N : 1) : cap);
+        const int64_t nvec = V / p.vec;
+        const int64_t nch = nvec > 0 ? (nvec + 1023) / 1024 : 1;
+        const int64_t want = (N * nch + 7) / 8;
+        const int64_t capb = (int64_t)sms * 12;
+        p.grid_bwd = (int)(want < capb ? (want > 0 ? want : 1) : capb);
+    }
+    return p;
+}
+
 ce_status ce_kl_forward(const void* student, const void* teacher, ce_dtype dt, ce_layout ls,
                         ce_layout lt, int64_t N, int64_t V, float* loss, float* lse_student,
                         float* lse_student_lo, float* lse_teacher, float* lse_teacher_lo,
@@ -502,7 +521,7 @@ ce_status ce_kl_forward(const void* student, const void* teacher, ce_dtype dt, c
             if (overlap(outs[i], outs[j])) return CE_EALIAS;
     }
     const bool vec_ok = vectorizable(student, Q, N, esz) && vectorizable(teacher, P, N, esz);
-    KlPlan p = plan_soft(N, V, esz, esz, vec_ok, device_sms(0));
+    KlPlan p = plan_kl(N, V, esz, vec_ok, device_sms(0));
     KlArgs a{};
     a.zq = student;
     a.zp = teacher;
@@ -547,7 +566,7 @@ ce_status ce_kl_backward(const float* grad_out, int64_t grad_stride, const void*
     if (lse_teacher_lo && overlap(ed, flat_extent(lse_teacher_lo, N, 4))) return CE_EALIAS;
     const bool vec_ok = vectorizable(student, Q, N, esz) && vectorizable(teacher, P, N, esz) &&
                         vectorizable(dstudent, D, N, dsz);
-    KlPlan p = plan_soft(N, V, esz, esz, vec_ok, device_sms(0));
+    KlPlan p = plan_kl(N, V, esz, vec_ok, device_sms(0));
     KlArgs a{};
     a.zq = student;
     a.zp = teacher;

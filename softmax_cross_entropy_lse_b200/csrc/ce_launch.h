@@ -136,6 +136,8 @@ struct SoftPlan {
     int vec;
     int G;
     int grid;
+    int cta;       // KL: long rows, too few of them for a warp each to fill the GPU
+    int grid_bwd;  // KL backward over (row, chunk) units
 };
 
 cudaError_t launch_soft_forward(const SoftPlan& p, const SoftArgs& a, int dz_t, int dt_t,

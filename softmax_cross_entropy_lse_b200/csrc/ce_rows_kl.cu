@@ -82,6 +82,25 @@ __device__ __forceinline__ void kl_group_reduce(KlState& st) {
     }
 }
 
+// loss and the two lse pairs of row r from its complete state
+__device__ __forceinline__ void kl_finalize(const KlArgs& a, const KlState& st, int64_t r) {
+    OnlineState oq = empty_state(), op = empty_state();
+    oq.m = st.mq;
+    oq.s = st.sq;
+    op.m = st.mp;
+    op.s = st.sp;
+    float Lq, hq, lq, Lp, hp, lp;
+    lse_pair(oq, Lq, hq, lq);
+    lse_pair(op, Lp, hp, lp);
+    a.lse_q[r] = hq;
+    a.lse_p[r] = hp;
+    if (a.lse_q_lo) a.lse_q_lo[r] = lq;
+    if (a.lse_p_lo) a.lse_p_lo[r] = lp;
+    float loss = __int_as_float(0x7fc00000);
+    if (isfinite(hq) && isfinite(hp)) loss = st.w / st.sp - (st.mp - st.mq) - (Lp - Lq);
+    a.loss[r] = loss;
+}
+
 template <typename T, int VEC, int G, int U, int MINB>
 __global__ void __launch_bounds__(256, MINB) k_kl_fwd(KlArgs a) {
     const T* __restrict__ zs = reinterpret_cast<const T*>(a.zq);
@@ -134,23 +153,7 @@ __global__ void __launch_bounds__(256, MINB) k_kl_fwd(KlArgs a) {
             }
         }
         kl_group_reduce<G>(st);
-        if (active && gl == 0) {
-            OnlineState oq = empty_state(), op = empty_state();
-            oq.m = st.mq;
-            oq.s = st.sq;
-            op.m = st.mp;
-            op.s = st.sp;
-            float Lq, hq, lq, Lp, hp, lp;
-            lse_pair(oq, Lq, hq, lq);
-            lse_pair(op, Lp, hp, lp);
-            a.lse_q[r] = hq;
-            a.lse_p[r] = hp;
-            if (a.lse_q_lo) a.lse_q_lo[r] = lq;
-            if (a.lse_p_lo) a.lse_p_lo[r] = lp;
-            float loss = __int_as_float(0x7fc00000);
-            if (isfinite(hq) && isfinite(hp)) loss = st.w / st.sp - (st.mp - st.mq) - (Lp - Lq);
-            a.loss[r] = loss;
-        }
+        if (active && gl == 0) kl_finalize(a, st, r);
     }
 }
 
@@ -216,6 +219,131 @@ __global__ void __launch_bounds__(256, MINB) k_kl_bwd(KlArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Long rows, few of them (the page's 512 x 151,936): a CTA of 8 warps per row
+// for the forward, the warp states meeting once in shared memory. The slots
+// alternate between two sets on successive rows, so no slot is rewritten
+// before every warp has passed the barrier of the row in between (the
+// slot-reuse race of "One barrier short" cannot occur).
+constexpr int kKlCtaWarps = 8;
+
+template <typename T, int VEC, int U, int MINB>
+__global__ void __launch_bounds__(kKlCtaWarps * 32, MINB) k_kl_fwd_cta(KlArgs a) {
+    __shared__ KlState slots[2][kKlCtaWarps];
+    const T* __restrict__ zs = reinterpret_cast<const T*>(a.zq);
+    const T* __restrict__ zt = reinterpret_cast<const T*>(a.zp);
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    constexpr int kThreads = kKlCtaWarps * 32;
+    const int64_t nvec = a.V / VEC;
+    const int tail = (int)(a.V - nvec * VEC);
+    int parity = 0;
+    for (int64_t r = blockIdx.x; r < a.N; r += gridDim.x, parity ^= 1) {
+        const T* qr = zs + row_offset(a.lq, r, a.N);
+        const T* pr = zt + row_offset(a.lp, r, a.N);
+        KlState st{-INFINITY, 0.f, -INFINITY, 0.f, 0.f};
+        for (int64_t vb = tid; vb < nvec; vb += (int64_t)kThreads * U) {
+            Raw<T, VEC> rq[U], rp[U];
+            bool ok[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t vi = vb + (int64_t)u * kThreads;
+                ok[u] = vi < nvec;
+                if (ok[u]) {
+                    load_raw<T, VEC>(qr, vi * VEC, a.lq.s_col, rq[u]);
+                    load_raw<T, VEC>(pr, vi * VEC, a.lp.s_col, rp[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (!ok[u]) continue;
+                float q[VEC], p[VEC];
+                unpack_raw<T, VEC>(rq[u], q);
+                unpack_raw<T, VEC>(rp[u], p);
+                kl_fold<VEC>(st, q, p);
+            }
+        }
+        for (int c = tid; c < tail; c += kThreads) {
+            const int64_t col = nvec * VEC + c;
+            const float q[1] = {to_f32(qr[col * a.lq.s_col])};
+            const float p[1] = {to_f32(pr[col * a.lp.s_col])};
+            kl_fold<1>(st, q, p);
+        }
+        kl_group_reduce<32>(st);
+        if (lane == 0) slots[parity][wid] = st;
+        __syncthreads();
+        if (wid == 0) {
+            st = slots[parity][lane & (kKlCtaWarps - 1)];
+            kl_group_reduce<kKlCtaWarps>(st);
+            if (lane == 0) kl_finalize(a, st, r);
+        }
+    }
+}
+
+// The backward needs no reduction: the rows are cut into chunks of
+// kKlChunkVecs vectors, one warp per (row, chunk) unit.
+constexpr int64_t kKlChunkVecs = 1024;
+
+template <typename T, typename TO, int VEC, int U, int MINB>
+__global__ void __launch_bounds__(256, MINB) k_kl_bwd_chunks(KlArgs a) {
+    const T* zs = reinterpret_cast<const T*>(a.zq);
+    const T* __restrict__ zt = reinterpret_cast<const T*>(a.zp);
+    TO* dz = reinterpret_cast<TO*>(a.dz);
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t nvec = a.V / VEC;
+    const int tail = (int)(a.V - nvec * VEC);
+    const int64_t nch = (nvec + kKlChunkVecs - 1) / kKlChunkVecs > 0 ? (nvec + kKlChunkVecs - 1) / kKlChunkVecs : 1;
+    for (int64_t unit = warp; unit < a.N * nch; unit += nwarps) {
+        const int64_t r = unit / nch;
+        const int64_t ch = unit - r * nch;
+        const T* qr = zs + row_offset(a.lq, r, a.N);
+        const T* pr = zt + row_offset(a.lp, r, a.N);
+        TO* dr = dz + row_offset(a.ld, r, a.N);
+        const float g = a.g[r * a.g_stride];
+        const float hq = a.lse_q[r], hp = a.lse_p[r];
+        const float cq = (a.lse_q_lo ? a.lse_q_lo[r] : 0.f) * kLog2e;
+        const float cp = (a.lse_p_lo ? a.lse_p_lo[r] : 0.f) * kLog2e;
+        const bool bad = !isfinite(hq) || !isfinite(hp);
+        const int64_t v1 = min(nvec, (ch + 1) * kKlChunkVecs);
+        for (int64_t vb = ch * kKlChunkVecs + lane; vb < v1; vb += (int64_t)32 * U) {
+            Raw<T, VEC> rq[U], rp[U];
+            bool ok[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t vi = vb + (int64_t)u * 32;
+                ok[u] = vi < v1;
+                if (ok[u]) {
+                    load_raw<T, VEC>(qr, vi * VEC, a.lq.s_col, rq[u]);
+                    load_raw<T, VEC>(pr, vi * VEC, a.lp.s_col, rp[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (!ok[u]) continue;
+                float q[VEC], p[VEC], o[VEC];
+                unpack_raw<T, VEC>(rq[u], q);
+                unpack_raw<T, VEC>(rp[u], p);
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    const float qe = ex2(fmaf(q[e] - hq, kLog2e, -cq));
+                    const float pe = ex2(fmaf(p[e] - hp, kLog2e, -cp));
+                    o[e] = bad ? __int_as_float(0x7fc00000) : g * (qe - pe);
+                }
+                store_vec<TO, VEC>(dr, (vb + (int64_t)u * 32) * VEC, a.ld.s_col, o);
+            }
+        }
+        if (ch == nch - 1) {
+            for (int c = lane; c < tail; c += 32) {
+                const int64_t col = nvec * VEC + c;
+                const float qe = ex2(fmaf(to_f32(qr[col * a.lq.s_col]) - hq, kLog2e, -cq));
+                const float pe = ex2(fmaf(to_f32(pr[col * a.lp.s_col]) - hp, kLog2e, -cp));
+                cvt_store1(dr + col * a.ld.s_col, bad ? __int_as_float(0x7fc00000) : g * (qe - pe));
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Four vectors of each row in flight per lane (eight on the scalar path) at
 // three blocks per SM: two rows' words take the registers of four blocks'
 // worth. The planner's lane grouping uses the same U.
@@ -227,6 +355,13 @@ template <int VEC, bool BWD = false> struct KlShape {
 template <typename T, int VEC>
 static cudaError_t kl_fwd_v(const KlPlan& p, const KlArgs& a, cudaStream_t s) {
     constexpr int U = KlShape<VEC>::U, MB = KlShape<VEC>::MINB;
+    if (p.cta) {
+        // four CTAs per SM for 4-byte rows: 592 rows in flight on a 148-SM
+        // part, so a batch of a few hundred long rows runs in one wave
+        // (16-bit rows need three CTAs' registers)
+        k_kl_fwd_cta<T, VEC, U, (VEC == 1 ? 2 : (VEC == 8 ? 3 : 4))><<<p.grid, kKlCtaWarps * 32, 0, s>>>(a);
+        return cudaGetLastError();
+    }
 #define CEB_KL(GG)                                                          \
     if (p.G == GG) {                                                        \
         k_kl_fwd<T, VEC, GG, U, MB><<<p.grid, 256, 0, s>>>(a);              \
@@ -240,6 +375,10 @@ static cudaError_t kl_fwd_v(const KlPlan& p, const KlArgs& a, cudaStream_t s) {
 template <typename T, typename TO, int VEC>
 static cudaError_t kl_bwd_v(const KlPlan& p, const KlArgs& a, cudaStream_t s) {
     constexpr int U = KlShape<VEC, true>::U, MB = KlShape<VEC, true>::MINB;
+    if (p.cta) {
+        k_kl_bwd_chunks<T, TO, VEC, U, MB><<<p.grid_bwd, 256, 0, s>>>(a);
+        return cudaGetLastError();
+    }
 #define CEB_KL(GG)                                                          \
     if (p.G == GG) {                                                        \
         k_kl_bwd<T, TO, VEC, GG, U, MB><<<p.grid, 256, 0, s>>>(a);          \
