@@ -83,14 +83,18 @@ def kernel_source_sha(files) -> str:
 
 def recorded_traffic(workload: str, kernel: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current sources of that pass's kernels; else None."""
+    the current sources of that pass's kernels (the entry's "sources", else
+    PASS_SOURCES); else None."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
-    if not os.path.exists(p) or kernel not in PASS_SOURCES:
+    if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(workload, {}).get(kernel)
-    if not e or e.get("source_sha") != kernel_source_sha(PASS_SOURCES[kernel]):
+    if not e:
+        return None
+    files = e.get("sources") or PASS_SOURCES.get(kernel)
+    if not files or e.get("source_sha") != kernel_source_sha(files):
         return None
     return e.get("bytes_per_launch")
 
@@ -490,7 +494,8 @@ def bench_soft(args, rk):
                 "h2d_bytes_per_step": 2 * N * V * 2, "d2h_bytes_per_step": 4 * N},
         "gpu_launches": 2 * args.steps,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 2), "peak": peak_hbm,
-                     "unit": "GB/s", "frac": round(achieved / peak_hbm, 4), "traffic": None,
+                     "unit": "GB/s", "frac": round(achieved / peak_hbm, 4),
+                     "traffic": recorded_traffic("soft", dom),
                      "peak_source": peak_src, "algorithmic_bytes_per_launch": dom_bytes},
     }
     clocks = clk.summary()
@@ -593,7 +598,8 @@ def bench_kl(args, rk):
                 "h2d_bytes_per_step": 2 * N * V * 4, "d2h_bytes_per_step": 4 * N},
         "gpu_launches": 2 * args.steps,
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 2), "peak": peak_hbm,
-                     "unit": "GB/s", "frac": round(achieved / peak_hbm, 4), "traffic": None,
+                     "unit": "GB/s", "frac": round(achieved / peak_hbm, 4),
+                     "traffic": recorded_traffic("kl", dom),
                      "peak_source": peak_src, "algorithmic_bytes_per_launch": dom_bytes},
     }
     clocks = clk.summary()
