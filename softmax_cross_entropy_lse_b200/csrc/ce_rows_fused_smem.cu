@@ -13,9 +13,11 @@
 //
 // A row longer than one CTA's share of shared memory is split across a
 // thread-block cluster of CL CTAs (CL = 1, 2, 4); CTA k holds vectors
-// [k S, (k+1) S) of the row. Each CTA reduces its slice, the CL partial
-// states are exchanged once through distributed shared memory, and every CTA
-// merges them in rank order, so all of them derive the same lse bits.
+// [k S, (k+1) S) of the row. Each CTA reduces its slice and pushes its state
+// into the shared memory of every other CTA of the cluster (st.async,
+// completed on the receiver's mbarrier, so no cluster-wide barrier or fence
+// runs per row); every CTA merges the CL states in rank order, so all of them
+// derive the same lse bits.
 //
 // Within a CTA, 8 warps own the 2 KB chunks of the slice round-robin (chunk c
 // belongs to warp c % 8). A warp's lane 0 copies its chunks in with 1-D bulk
@@ -40,12 +42,17 @@ constexpr int kSmChunkVecs = 128;  // 16-byte vectors per 2 KB chunk
 constexpr int kSmMaxChunks = kSmemRowMaxChunks;
 static_assert(kSmMaxChunks <= 8 * 32, "per-warp chunk masks are 32 bits");
 
-struct __align__(8) StateRec {
-    float m, s, t;
-    int k;
-    float av;
-    int ai;
-};
+// Pushes 16 bytes into the shared memory of another CTA of the cluster
+// (remote_addr from mapa) and counts them on that CTA's mbarrier (remote_bar,
+// from mapa too) as transaction bytes: the receiver learns of the data from
+// its own barrier, with no cluster-wide fence.
+__device__ __forceinline__ void st_async_v4(uint32_t remote_addr, const uint4& v, uint32_t remote_bar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+            remote_addr),
+        "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(remote_bar)
+        : "memory");
+}
 
 template <typename TI, bool ARGMAX, bool WITH_T>
 __device__ __forceinline__ void fold_chunk(OnlineState& st, const uint4* buf, int nvc, int lane,
@@ -140,7 +147,10 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
     extern __shared__ __align__(128) uint8_t row_smem[];
     __shared__ __align__(8) uint64_t full_bar[kSmMaxChunks];
     __shared__ OnlineState wslot[2][kSmWarps];
-    __shared__ StateRec cslot[2];
+    // CTA states of the cluster, pushed by their owners: [row parity][source
+    // rank][two 16-byte words], completed on xbar[row parity]
+    __shared__ __align__(16) uint4 xslot[2][4][2];
+    __shared__ __align__(8) uint64_t xbar[2];
     __shared__ int abort_flag;
 
     const TI* z = reinterpret_cast<const TI*>(a.z);
@@ -161,9 +171,15 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
 
     if (lane == 0)
         for (int c = wid; c < nch; c += kSmWarps) mbar_init(smem_u32(&full_bar[c]), 1);
-    if (tid == 0) abort_flag = 0;
+    if (tid == 0) {
+        abort_flag = 0;
+        mbar_init(smem_u32(&xbar[0]), 1);
+        mbar_init(smem_u32(&xbar[1]), 1);
+    }
     if (lane == 0) mbar_fence_init();
     __syncthreads();
+    // every CTA's barriers exist before any peer pushes a state into them
+    if constexpr (CL > 1) cluster_sync();
 
     auto chunk_vecs = [&](int c) { return min(kSmChunkVecs, nv - c * kSmChunkVecs); };
     auto chunk_buf = [&](int c) { return reinterpret_cast<const uint4*>(row_smem + (size_t)c * 2048); };
@@ -228,19 +244,37 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
         st = wslot[par][lane & (kSmWarps - 1)];
         group_reduce<kSmWarps, ARGMAX, WITH_T>(st);
         if constexpr (CL > 1) {
+            // push this CTA's state into every peer's slot [par][rank]; wait
+            // for the peers' states on this CTA's own barrier. A peer writes
+            // slot [par] again only for row it + 2, after it has received this
+            // CTA's state of row it + 1, which this CTA sends after reading
+            // the slots of row it: no slot is overwritten before it is read.
+            const uint32_t bar = smem_u32(&xbar[par]);
             if (tid == 0) {
-                StateRec rec{st.m, st.s, st.t, st.k, st.av, st.ai};
-                cslot[par] = rec;
+                mbar_expect_tx(bar, (uint32_t)(CL - 1) * 32u);
+                const uint4 w0 = make_uint4(__float_as_uint(st.m), __float_as_uint(st.s),
+                                            __float_as_uint(st.t), (uint32_t)st.k);
+                const uint4 w1 = make_uint4(__float_as_uint(st.av), (uint32_t)st.ai, 0u, 0u);
+                const uint32_t src = smem_u32(&xslot[par][rank][0]);
+#pragma unroll
+                for (uint32_t k = 0; k < (uint32_t)CL; ++k) {
+                    if (k == rank) continue;
+                    const uint32_t ra = mapa_shared(src, k), rb = mapa_shared(bar, k);
+                    st_async_v4(ra, w0, rb);
+                    st_async_v4(ra + 16, w1, rb);
+                }
             }
-            cluster_sync();
-            const uint32_t ra = mapa_shared(smem_u32(&cslot[par]), (uint32_t)(lane & (CL - 1)));
-            const uint2 p0 = ld_cluster_v2(ra), p1 = ld_cluster_v2(ra + 8), p2 = ld_cluster_v2(ra + 16);
-            st.m = __uint_as_float(p0.x);
-            st.s = __uint_as_float(p0.y);
-            st.t = __uint_as_float(p1.x);
-            st.k = (int)p1.y;
-            st.av = __uint_as_float(p2.x);
-            st.ai = (int)p2.y;
+            if (!dead && !mbar_wait(bar, (uint32_t)(it >> 1) & 1u, &abort_flag)) dead = true;
+            const uint32_t from = (uint32_t)(lane & (CL - 1));
+            if (from != rank) {
+                const uint4 w0 = xslot[par][from][0], w1 = xslot[par][from][1];
+                st.m = __uint_as_float(w0.x);
+                st.s = __uint_as_float(w0.y);
+                st.t = __uint_as_float(w0.z);
+                st.k = (int)w0.w;
+                st.av = __uint_as_float(w1.x);
+                st.ai = (int)w1.y;
+            }
             group_reduce<CL, ARGMAX, WITH_T>(st);
         }
         if (rank == 0 && tid == 0) finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);
@@ -290,7 +324,7 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
         for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps)
             if ((pend >> i) & 1u) mbar_wait(smem_u32(&full_bar[c]), (phase >> i) & 1u, &never);
     }
-    // no CTA leaves while another may still read its exchange slot
+    // no CTA leaves while a peer may still push into its slots
     if constexpr (CL > 1) cluster_sync();
 }
 
