@@ -248,8 +248,9 @@ __global__ void __launch_bounds__(kCtaThreads, kCtaMinBlocks) k_fwd_cta(FwdArgs 
 // short" cannot occur), and the warps of a CTA stay within two units of each
 // other, streaming neighbouring parts of the same rows.
 constexpr int kRingWarps = 8;
-constexpr int kRingStages = 4;
-constexpr int kRingVecs = 128;  // 2 KB per stage
+constexpr int kRingStages = 2;
+constexpr int kRingVecs = 256;  // 4 KB per stage
+constexpr int kRingPart = 128;  // vectors folded at a time (4 per lane)
 constexpr size_t kRingSmem = (size_t)kRingWarps * kRingStages * kRingVecs * 16;
 static_assert((kRingStages & (kRingStages - 1)) == 0 && (kRingWarps & (kRingWarps - 1)) == 0,
               "stage and warp counts are powers of two");
@@ -313,7 +314,7 @@ template <typename T, bool ARGMAX, bool WITH_T>
 __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
     using namespace sm100;
     constexpr int VEC = ElemTraits<T>::kVec;
-    constexpr int kPerLane = kRingVecs / 32;
+    constexpr int kPerLane = kRingPart / 32;
     extern __shared__ __align__(128) uint8_t ring_smem[];
     __shared__ __align__(8) uint64_t full_bar[kRingWarps][kRingStages];
     __shared__ OnlineState slots[2][kRingWarps];
@@ -334,8 +335,8 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
     // prologue: the first kRingStages chunks of this warp's sequence
     RingCursor<T> iss;
     iss.start(a, units, nvec, wid);
-    // 32-bit counters: stage = count % 4 and parity = (count / 4) % 2 stay
-    // exact across wraparound (4 and 8 divide 2^32)
+    // 32-bit counters: stage = count % kRingStages and parity = (count /
+    // kRingStages) % 2 stay exact across wraparound (powers of two divide 2^32)
     uint32_t issued = 0;
     for (int q = 0; q < kRingStages && iss.valid(units); ++q) {
         if (lane == 0) {
@@ -378,38 +379,44 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
             if (!dead) {
                 const int64_t left = ru.nv - (int64_t)j * kRingVecs;
                 const int nvc = (int)(left < kRingVecs ? left : kRingVecs);
-                const uint4* buf = reinterpret_cast<const uint4*>(ring + stage * kRingVecs * 16);
-                if constexpr (sizeof(T) == 2 && !ARGMAX) {
-                    // raw 16-bit words: packed max, widened pairwise for the sum
-                    uint4 w[kPerLane];
-                    bool ok[kPerLane];
+                // the chunk is folded in parts of kRingPart vectors (4 per lane)
+#pragma unroll 1
+                for (int h = 0; h < kRingVecs / kRingPart && h * kRingPart < nvc; ++h) {
+                    const uint4* buf =
+                        reinterpret_cast<const uint4*>(ring + stage * kRingVecs * 16) + h * kRingPart;
+                    const int nvh = min(kRingPart, nvc - h * kRingPart);
+                    if constexpr (sizeof(T) == 2 && !ARGMAX) {
+                        // raw 16-bit words: packed max, widened pairwise for the sum
+                        uint4 w[kPerLane];
+                        bool ok[kPerLane];
 #pragma unroll
-                    for (int q = 0; q < kPerLane; ++q) {
-                        const int vi = q * 32 + lane;
-                        ok[q] = vi < nvc;
-                        if (ok[q]) w[q] = buf[vi];
-                    }
-                    if (nvc == kRingVecs)
-                        fold_raw16<T, kPerLane, false, WITH_T>(st, w, ok);
-                    else
-                        fold_raw16<T, kPerLane, true, WITH_T>(st, w, ok);
-                } else {
-                    float v[kPerLane][VEC];
-                    bool ok[kPerLane];
-                    int c0[kPerLane];
-#pragma unroll
-                    for (int q = 0; q < kPerLane; ++q) {
-                        const int vi = q * 32 + lane;
-                        ok[q] = vi < nvc;
-                        c0[q] = (int)((ru.v0 + (int64_t)j * kRingVecs + vi) * VEC);
-                        if (ok[q]) unpack_words<T>(buf[vi], v[q]);
-                    }
-                    if (nvc == kRingVecs) {
-                        fold_vecs<kPerLane, VEC, false>(st, v, ok);
-                        if constexpr (ARGMAX) argmax_vecs<kPerLane, VEC, false>(st, v, ok, c0);
+                        for (int q = 0; q < kPerLane; ++q) {
+                            const int vi = q * 32 + lane;
+                            ok[q] = vi < nvh;
+                            if (ok[q]) w[q] = buf[vi];
+                        }
+                        if (nvh == kRingPart)
+                            fold_raw16<T, kPerLane, false, WITH_T>(st, w, ok);
+                        else
+                            fold_raw16<T, kPerLane, true, WITH_T>(st, w, ok);
                     } else {
-                        fold_vecs<kPerLane, VEC, true>(st, v, ok);
-                        if constexpr (ARGMAX) argmax_vecs<kPerLane, VEC, true>(st, v, ok, c0);
+                        float v[kPerLane][VEC];
+                        bool ok[kPerLane];
+                        int c0[kPerLane];
+#pragma unroll
+                        for (int q = 0; q < kPerLane; ++q) {
+                            const int vi = q * 32 + lane;
+                            ok[q] = vi < nvh;
+                            c0[q] = (int)((ru.v0 + (int64_t)j * kRingVecs + h * kRingPart + vi) * VEC);
+                            if (ok[q]) unpack_words<T>(buf[vi], v[q]);
+                        }
+                        if (nvh == kRingPart) {
+                            fold_vecs<kPerLane, VEC, false>(st, v, ok);
+                            if constexpr (ARGMAX) argmax_vecs<kPerLane, VEC, false>(st, v, ok, c0);
+                        } else {
+                            fold_vecs<kPerLane, VEC, true>(st, v, ok);
+                            if constexpr (ARGMAX) argmax_vecs<kPerLane, VEC, true>(st, v, ok, c0);
+                        }
                     }
                 }
             }
