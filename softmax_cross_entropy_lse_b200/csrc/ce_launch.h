@@ -49,7 +49,6 @@ cudaError_t launch_forward(const FwdPlan& p, const FwdArgs& a, int dtype, cudaSt
 
 // rows per lane per step of the tiny-row forward
 constexpr int kTinyRows = 2;
-int cta_threads_forward();
 
 // ---- row backward ------------------------------------------------------------
 struct BwdArgs {

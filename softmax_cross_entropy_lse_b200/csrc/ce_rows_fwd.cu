@@ -607,6 +607,4 @@ cudaError_t launch_forward(const FwdPlan& p, const FwdArgs& a, int dtype, cudaSt
     return cudaErrorInvalidValue;
 }
 
-int cta_threads_forward() { return kCtaThreads; }
-
 }  // namespace ceb
