@@ -156,6 +156,13 @@ static FwdPlan plan_forward(int64_t N, int64_t V, int esz, bool vec_ok, int sms)
         const int64_t want = (N + rows_per_block - 1) / rows_per_block;
         const int64_t cap = (int64_t)sms * 16;
         p.grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
+        // whole-vector 4-byte rows that one step covers: pipelined through
+        // shared memory, three resident blocks per SM, every block resident
+        if (vec_ok && esz == 4 && p.G >= 2 && V % p.vec == 0 && nvec <= (int64_t)p.G * 8) {
+            p.pipe = 1;
+            const int64_t capp = (int64_t)sms * 3;
+            p.grid = (int)(want < capp ? (want > 0 ? want : 1) : capp);
+        }
         return p;
     }
     p.kind = FwdPlan::kCta;

@@ -39,6 +39,7 @@ struct FwdPlan {
     int G, U;       // packed: lanes per row, vectors per lane per step; tiny: U vectors per row
     int R;          // packed: rows per group per step
     int ring;       // long rows through per-warp bulk-copy rings
+    int pipe;       // packed 4-byte rows of one step, pipelined through shared memory
     int grid;
     int merge_grid;
     int splits;

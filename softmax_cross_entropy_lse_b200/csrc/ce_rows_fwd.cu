@@ -87,6 +87,88 @@ __global__ void __launch_bounds__(256, MINB) k_fwd_packed(FwdArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Packed rows that one step covers (nvec <= G U, whole 16-byte vectors, no
+// tail), pipelined across row groups: while a warp folds its current group
+// of 32/G rows, the next group's vectors are already streaming into its
+// shared-memory slot (cp.async, two stages per warp). Each lane reads back
+// only the slots it filled, so no barrier is needed and the slot layout
+// [u][lane] is free of bank conflicts.
+constexpr int kPipeWarps = 8;
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sm100::smem_u32(smem)),
+                 "l"(reinterpret_cast<uint64_t>(gmem))
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int n>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(n) : "memory");
+}
+
+template <typename T, int VEC, int G, int U, bool ARGMAX, int MINB>
+__global__ void __launch_bounds__(kPipeWarps * 32, MINB) k_fwd_packed_pipe(FwdArgs a) {
+    extern __shared__ __align__(16) uint4 pipe_smem[];  // [2][kPipeWarps][U][32]
+    const T* __restrict__ z = reinterpret_cast<const T*>(a.z);
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int gl = lane & (G - 1);
+    constexpr int kRowsPerStep = 32 / G;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t step = nwarps * kRowsPerStep;
+    const int64_t nvec = a.V / VEC;
+    const RowOut out{a.loss, a.lse, a.lse_lo, a.argmax, a.err};
+    auto slot = [&](int s, int u) { return pipe_smem + ((s * kPipeWarps + wid) * U + u) * 32 + lane; };
+    auto issue = [&](int64_t base, int s) {
+        const int64_t r = base + lane / G;
+        if (r < a.N) {
+            const T* row = z + row_offset(a.lz, r, a.N);
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t vi = u * G + gl;
+                if (vi < nvec) cp_async16(slot(s, u), row + vi * VEC);
+            }
+        }
+        cp_async_commit();  // one group per row group, empty or not
+    };
+
+    int s = 0;
+    int64_t base = warp * kRowsPerStep;
+    if (base < a.N) issue(base, 0);
+    for (; base < a.N; base += step, s ^= 1) {
+        issue(base + step, s ^ 1);
+        const int64_t r = base + lane / G;
+        const bool active = r < a.N;
+        int64_t y = a.ignore;
+        float zy = 0.f;
+        if (active) {
+            const T* row = z + row_offset(a.lz, r, a.N);
+            y = load_target(a.y, a.tdt, row_offset(a.ly, r, a.N));
+            if (gl == 0 && y >= 0 && y < a.V && y != a.ignore) zy = to_f32(row[y * a.lz.s_col]);
+        }
+        cp_async_wait<1>();  // this row group's copies have landed
+        OnlineState st = empty_state();
+        if (active) {
+            float v[U][VEC];
+            bool ok[U];
+            int c0[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t vi = u * G + gl;
+                ok[u] = vi < nvec;
+                c0[u] = (int)(vi * VEC);
+                if (ok[u]) unpack_words<T>(*slot(s, u), v[u]);
+            }
+            fold_vecs<U, VEC, true>(st, v, ok);
+            if constexpr (ARGMAX) argmax_vecs<U, VEC, true>(st, v, ok, c0);
+        }
+        group_reduce<G, ARGMAX>(st);
+        if (active && gl == 0) finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);
+    }
+    cp_async_wait<0>();
+}
+
+// ---------------------------------------------------------------------------
 // Tiny rows: one or two 16-byte vectors and no ragged tail (for instance 8
 // floats). One lane per row and R rows per lane per step, with every load of
 // the step issued before any is used. The whole row sits in registers, so it
@@ -557,6 +639,28 @@ static cudaError_t launch_ring(const FwdPlan& p, const FwdArgs& a, cudaStream_t 
     return cudaGetLastError();
 }
 
+template <typename T, int VEC>
+static cudaError_t launch_pipe(const FwdPlan& p, const FwdArgs& a, cudaStream_t s) {
+    constexpr int U = 8;
+    constexpr size_t smem = (size_t)2 * kPipeWarps * U * 32 * 16;  // 64 KB
+#define CEB_PIPE(GG)                                                                            \
+    if (p.G == GG) {                                                                            \
+        static bool attr = false;                                                               \
+        if (!attr) {                                                                            \
+            cudaError_t e = cudaFuncSetAttribute(k_fwd_packed_pipe<T, VEC, GG, U, false, 3>,     \
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,   \
+                                                 (int)smem);                                    \
+            if (e != cudaSuccess) return e;                                                     \
+            attr = true;                                                                        \
+        }                                                                                       \
+        k_fwd_packed_pipe<T, VEC, GG, U, false, 3><<<p.grid, kPipeWarps * 32, smem, s>>>(a);    \
+        return cudaGetLastError();                                                              \
+    }
+    CEB_PIPE(2) CEB_PIPE(4) CEB_PIPE(8) CEB_PIPE(16) CEB_PIPE(32)
+#undef CEB_PIPE
+    return cudaErrorInvalidValue;
+}
+
 template <typename T, bool ARGMAX, bool WITH_T>
 static cudaError_t launch_tiny(const FwdPlan& p, const FwdArgs& a, cudaStream_t s) {
     constexpr int V8 = ElemTraits<T>::kVec;
@@ -573,6 +677,10 @@ static cudaError_t launch_fwd_t(const FwdPlan& p, const FwdArgs& a, cudaStream_t
     constexpr int V8 = ElemTraits<T>::kVec;
     if (p.kind == FwdPlan::kTiny)
         return a.eps != 0.f ? launch_tiny<T, ARGMAX, true>(p, a, s) : launch_tiny<T, ARGMAX, false>(p, a, s);
+    if constexpr (sizeof(T) == 4 && !ARGMAX) {
+        // (with argmax, the plain packed kernel below takes the same plan)
+        if (p.kind == FwdPlan::kPacked && p.pipe) return launch_pipe<T, V8>(p, a, s);
+    }
     if (p.kind == FwdPlan::kPacked) {
         return p.vec == 1 ? launch_packed<T, 1, ARGMAX>(a, p.G, p.U, p.grid, s)
                           : launch_packed<T, V8, ARGMAX>(a, p.G, p.U, p.grid, s);
