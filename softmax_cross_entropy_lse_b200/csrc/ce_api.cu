@@ -205,6 +205,19 @@ static BwdPlan plan_backward(int64_t N, int64_t V, int esz_in, bool vec_ok, int 
     p.ring = 0;
     p.rows = 0;
     const int kU = p.vec == 1 ? 8 : 32 / p.vec;
+    if (vec_ok && V % p.vec == 0 && nvec <= 2) {
+        // one or two whole vectors per row: a lane per row, every block resident
+        p.tiny = 1;
+        p.G = 1;
+        p.U = (int)nvec;
+        *nchunks = 1;
+        *vpc = nvec;
+        const int64_t rows_per_block = 256 * (int64_t)kTinyRows;
+        const int64_t want = (N + rows_per_block - 1) / rows_per_block;
+        const int64_t cap = (int64_t)sms * (p.U == 1 ? 4 : 3);
+        p.grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
+        return p;
+    }
     if (nvec <= 256) {
         p.rows = 1;
         p.G = packed_lanes(nvec);

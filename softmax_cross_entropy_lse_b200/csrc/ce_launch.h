@@ -76,6 +76,7 @@ struct BwdPlan {
     int R;     // units per group per step
     int ring;  // long rows through per-warp bulk-copy rings
     int rows;  // short rows, one unit per row (k_bwd_rows)
+    int tiny;  // one or two whole vectors per row: a lane per row (k_bwd_tiny)
     int grid;
 };
 

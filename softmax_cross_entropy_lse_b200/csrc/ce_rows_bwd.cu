@@ -155,6 +155,75 @@ __global__ void __launch_bounds__(256) k_bwd(BwdArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Tiny rows (one or two 16-byte vectors, no ragged tail): one lane per row
+// and R rows per lane per step, with every load of the step issued before
+// any is used, and the warp's next step of rows sent into L2 ahead of time
+// when the rows lie back to back. The gradient is the one k_bwd_rows forms.
+template <typename TI, typename TO, int NV, int R, int MINB>
+__global__ void __launch_bounds__(256, MINB) k_bwd_tiny(BwdArgs a) {
+    constexpr int VEC = ElemTraits<TI>::kVec;
+    constexpr int n = NV * VEC;
+    const TI* z = reinterpret_cast<const TI*>(a.z);
+    TO* dz = reinterpret_cast<TO*>(a.dz);
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const float inv_v = 1.f / (float)a.V;
+    const float nan = __int_as_float(0x7fc00000);
+    const bool dense = a.lz.inner >= a.N && a.lz.s_inner == (int64_t)n;
+
+    for (int64_t base = warp * 32 * R; base < a.N; base += nwarps * 32 * R) {
+        if (dense && lane == 0) {
+            const int64_t bn = base + nwarps * 32 * R;
+            if (bn < a.N) {
+                const int64_t rows = min((int64_t)32 * R, a.N - bn);
+                sm100::bulk_prefetch_l2(z + bn * n, (uint32_t)(rows * n * sizeof(TI)));
+            }
+        }
+        uint4 w[R][NV];
+        int64_t y[R];
+        float hi[R], lo[R], g[R];
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            const int64_t r = base + 32 * k + lane;
+            y[k] = a.ignore;
+            hi[k] = lo[k] = g[k] = 0.f;
+            if (r < a.N) {
+                const TI* row = z + row_offset(a.lz, r, a.N);
+                y[k] = load_target(a.y, a.tdt, row_offset(a.ly, r, a.N));
+                hi[k] = a.lse[r];
+                lo[k] = a.lse_lo ? a.lse_lo[r] : 0.f;
+                g[k] = a.g[r * a.g_stride];
+#pragma unroll
+                for (int v = 0; v < NV; ++v) w[k][v] = *(reinterpret_cast<const uint4*>(row) + v);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            const int64_t r = base + 32 * k + lane;
+            if (r >= a.N) continue;
+            const bool zero = y[k] == a.ignore;
+            const bool bad = !zero && (y[k] < 0 || y[k] >= a.V);
+            const int yc = (zero || bad) ? -1 : (int)y[k];  // column of the target, if any
+            const float c_lo = lo[k] * kLog2e, c_eps = g[k] * a.eps * inv_v, c_tgt = g[k] * (1.f - a.eps);
+            TO* drow = dz + row_offset(a.ld, r, a.N);
+#pragma unroll
+            for (int v = 0; v < NV; ++v) {
+                float x[VEC], o[VEC];
+                unpack_words<TI>(w[k][v], x);
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    const float p = ex2(fmaf(x[e] - hi[k], kLog2e, -c_lo));
+                    o[e] = (zero || bad) ? (bad ? nan : 0.f) : fmaf(g[k], p, -c_eps);
+                    if (yc == v * VEC + e) o[e] -= c_tgt;
+                }
+                store_vec<TO, VEC>(drow, v * VEC, 1, o);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Short rows: G lanes per row, 32/G rows per warp, U vectors per lane per
 // step. Every load of a row (target, lse pair, g and the logits of the first
 // step) is issued before any of them is used, so a group waits on memory
@@ -502,6 +571,14 @@ static cudaError_t launch_bwd_rows(const BwdPlan& p, const BwdArgs& a, cudaStrea
 
 template <typename TI, typename TO>
 static cudaError_t launch_bwd_t(const BwdPlan& p, const BwdArgs& a, cudaStream_t s) {
+    if (p.tiny) {
+        // register budgets: 64 per thread for one vector per row, 85 for two
+        if (p.U == 1)
+            k_bwd_tiny<TI, TO, 1, kTinyRows, 4><<<p.grid, 256, 0, s>>>(a);
+        else
+            k_bwd_tiny<TI, TO, 2, kTinyRows, 3><<<p.grid, 256, 0, s>>>(a);
+        return cudaGetLastError();
+    }
     if (p.ring) return launch_bwd_ring<TI, TO>(p, a, s);
     if (p.rows) {
         if (p.vec == 1) return launch_bwd_rows<TI, TO, 1>(p, a, s);

@@ -398,6 +398,26 @@ def test_tiny_rows_strided_view_matches_copy(orc):
     check_rows(orc, r1, d1, z64, t[:, 1:].reshape(-1), 0.1, -100, "f32", "f32")
 
 
+@pytest.mark.parametrize("V,dt", [(4, "f32"), (8, "f32"), (16, "bf16")])
+def test_tiny_rows_backward_per_row_g_and_in_place(orc, V, dt):
+    """Tiny-row VJP with a per-row upstream gradient read through a strided
+    view, and written over the logits it reads."""
+    N = 3001
+    z, z32, y = wl.rows(N, V, dt, seed=40 + V, std=2.0, ignore_frac=0.1)
+    g = np.random.default_rng(V).uniform(-1.0, 1.0, N).astype(np.float32)
+    zt, yt = upload(z, dt), upload(y)
+    r = ce.ce_forward(zt, yt, 0.1)
+    g2 = upload(np.repeat(g, 3))[::3]
+    dz = ce.ce_backward(g2, zt, yt, r.lse, r.lse_lo, 0.1)
+    torch.cuda.synchronize()
+    ref = orc.ce_backward(z32.astype(np.float64), y, g.astype(np.float64), 0.1)
+    assert_grad_close(f32(dz), ref, dt, dt)
+    out = ce.ce_backward(g2, zt, yt, r.lse, r.lse_lo, 0.1, dlogits=zt)
+    torch.cuda.synchronize()
+    assert out.data_ptr() == zt.data_ptr()
+    assert torch.equal(zt, dz)
+
+
 def test_tiny_rows_forward_matches_fused():
     z, _, y = wl.rows(5000, 8, "f32", seed=2, ignore_frac=0.1)
     zt, yt = upload(z), upload(y)
