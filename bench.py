@@ -692,6 +692,7 @@ def bench_linear(args, rk):
         "data": "synthetic",
         "fwd_tflops": round(fwd_flop / (fwd_ms * 1e-3) / 1e12, 2), "fwd_ms": round(fwd_ms, 4),
         "bwd_ms": round(bwd_ms, 4),
+        "workspace_bytes": {"forward": int(ws_f.numel()), "backward": int(ws_b.numel())},
         "config": {"workload": f"c5: fused linear CE, H ({N}, {D}) bf16 ~N(0,1), W ({V}, {D}) "
                                "bf16 ~N(0, std 0.02), forward + backward (logits recomputed)",
                    "N": N, "V": V, "D": D, "flop_per_step": step_flop,
@@ -699,7 +700,7 @@ def bench_linear(args, rk):
                    "parallelism": f"rows sharded over {world} rank(s), no data-path collective"},
         "e2e": {"value": round(world * step_flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": (N * D + V * D) * 2 + 4 * N, "d2h_bytes_per_step": 4 * N},
-        "gpu_launches": (2 + 2 + 3 * ((V + 8191) // 8192)) * args.steps,
+        "gpu_launches": (2 + 1 + 4 * ((V + 8191) // 8192)) * args.steps,
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2),
                      "peak": peak_sust, "unit": "TFLOP/s", "frac": round(achieved / peak_sust, 4),
                      "traffic": recorded_traffic("c5", dom), "peak_source": src + " (sustained)"},

@@ -541,8 +541,8 @@ struct BwdLayout {
 static BwdLayout bwd_layout(int64_t N, int64_t V, int64_t D) {
     BwdLayout L{};
     L.ld_ht = round_up(N, 8);
-    L.ld_wt = round_up(V, 8);
     L.vc = V < kBwdChunk ? round_up(V, kBN) : kBwdChunk;
+    L.ld_wt = L.vc;  // one vocabulary chunk of W^T at a time
     L.ld_gt = round_up(N, 8);
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -551,7 +551,7 @@ static BwdLayout bwd_layout(int64_t N, int64_t V, int64_t D) {
         return o;
     };
     L.off_ht = take((size_t)D * L.ld_ht * 2);
-    L.off_wt = take((size_t)D * L.ld_wt * 2);
+    L.off_wt = take((size_t)D * L.vc * 2);
     L.off_g = take((size_t)N * L.vc * 2);
     L.off_gt = take((size_t)L.vc * L.ld_gt * 2);
     L.off_acc = take((size_t)N * D * 4);
@@ -649,25 +649,31 @@ ce_status linear_ce_backward(const float* grad_out, int64_t grad_stride, const v
     auto* GT = reinterpret_cast<__nv_bfloat16*>(ws + L.off_gt);
     float* dH_acc = dH_dt == CE_F32 ? static_cast<float*>(dH) : reinterpret_cast<float*>(ws + L.off_acc);
 
-    // transposed copies of H and W (K-major operands of the dW and dH passes)
+    // transposed copy of H (the K-major B operand of the dW pass); W is
+    // transposed one vocabulary chunk at a time below
     {
         const int64_t t1 = ((N + 63) / 64) * ((D + 63) / 64);
-        const int64_t t2 = ((V + 63) / 64) * ((D + 63) / 64);
         k_transpose_bf16<<<(int)(t1 < (int64_t)sms * 8 ? t1 : (int64_t)sms * 8), 256, 0, s>>>(
             static_cast<const __nv_bfloat16*>(H), ld_h, HT, L.ld_ht, N, D);
-        k_transpose_bf16<<<(int)(t2 < (int64_t)sms * 8 ? t2 : (int64_t)sms * 8), 256, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(W), ld_w, WT, L.ld_wt, V, D);
         if (cudaGetLastError() != cudaSuccess) return CE_ECUDA;
     }
-    CUtensorMap mH, mW, mHT, mWT;
-    if (!make_map(&mH, H, N, D, ld_h, kBM) || !make_map(&mW, W, V, D, ld_w, kBN) ||
-        !make_map(&mHT, HT, D, N, L.ld_ht, kBN) || !make_map(&mWT, WT, D, V, L.ld_wt, kBN))
+    CUtensorMap mH, mHT;
+    if (!make_map(&mH, H, N, D, ld_h, kBM) || !make_map(&mHT, HT, D, N, L.ld_ht, kBN))
         return CE_ECUDA;
 
     const int64_t nchunks = (V + L.vc - 1) / L.vc;
     for (int64_t c = 0; c < nchunks; ++c) {
         const int64_t v0 = c * L.vc;
         const int64_t vcv = (V - v0) < L.vc ? (V - v0) : L.vc;  // valid columns
+        // W_c^T (D x vcv, leading dimension vc): the K-major B operand of the
+        // dH pass. Stream order keeps the previous chunk's dH pass ahead of
+        // this overwrite.
+        {
+            const int64_t t2 = ((vcv + 63) / 64) * ((D + 63) / 64);
+            k_transpose_bf16<<<(int)(t2 < (int64_t)sms * 8 ? t2 : (int64_t)sms * 8), 256, 0, s>>>(
+                static_cast<const __nv_bfloat16*>(W) + v0 * ld_w, ld_w, WT, L.ld_wt, vcv, D);
+            if (cudaGetLastError() != cudaSuccess) return CE_ECUDA;
+        }
         // GEMM 1: Z_c = H W_c^T, epilogue writes G_c and G_c^T
         {
             CUtensorMap mWc;
@@ -710,16 +716,17 @@ ce_status linear_ce_backward(const float* grad_out, int64_t grad_stride, const v
             a.c_f32 = dW_dt == CE_F32;
             if (launch_gemm<kEpiStore>(mGT, mHT, a, sms, s) != cudaSuccess) return CE_ECUDA;
         }
-        // GEMM 3: dH (+)= G_c W_c  (A = G_c, B = W^T columns [v0, v0+vcv), K = vcv)
+        // GEMM 3: dH (+)= G_c W_c  (A = G_c, B = W_c^T, K = vcv)
         {
-            CUtensorMap mG;
-            if (!make_map(&mG, G, N, vcv, L.vc, kBM)) return CE_ECUDA;
+            CUtensorMap mG, mWT;
+            if (!make_map(&mG, G, N, vcv, L.vc, kBM) || !make_map(&mWT, WT, D, vcv, L.ld_wt, kBN))
+                return CE_ECUDA;
             GemmArgs a{};
             a.M = (int)N;
             a.Nn = (int)D;
             a.K = (int)vcv;
             a.kA0 = 0;
-            a.kB0 = (int)v0;
+            a.kB0 = 0;
             a.tiles_per_unit = 1;
             a.err = err;
             a.acc = dH_acc;
