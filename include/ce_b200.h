@@ -68,7 +68,8 @@ typedef enum {
     CE_EWORKSPACE = 3, /* workspace missing or smaller than the *_workspace_size query */
     CE_ECUDA = 4,      /* a CUDA runtime call failed (launch, attribute query) */
     CE_ETARGET = 5,    /* device flag: a target outside [0, V) that is not ignore_index */
-    CE_ENOTSUP = 6     /* a configuration this build does not implement */
+    CE_ENOTSUP = 6,    /* a configuration this build does not implement */
+    CE_ETIMEOUT = 7    /* device flag: a kernel gave up a bounded wait (outputs invalid) */
 } ce_status;
 
 /* ------------------------------------------------------------------------ *
@@ -284,10 +285,11 @@ ce_status linear_ce_backward(const float* grad_out, int64_t grad_stride,
 /* ------------------------------------------------------------------------ *
  * Forward without a caller-provided workspace.
  * The pages have no counterpart to this call; it exists for callers that
- * cannot allocate device memory or pass a workspace: code running while a
- * stream is being captured into a CUDA graph (allocation is refused there),
- * plugin hosts that own all device memory through their own pool, and C
- * callers without an allocator.
+ * cannot allocate device memory or pass a workspace: plugins inside a host
+ * application that owns all device memory through its own pool (a raw
+ * allocation would bypass its accounting), loops with a memory budget fixed
+ * at start-up that must not run out of memory halfway, and C callers without
+ * an allocator (cudaMalloc may also synchronise the device).
  *
  * Same arguments, results and errors as ce_forward, without workspace and
  * ws_bytes. The scratch for the vocabulary split lives in a library-owned
@@ -317,9 +319,31 @@ ce_status ce_forward_noalloc(const void* logits, ce_dtype dt, ce_layout lg,
 /* ------------------------------------------------------------------------ */
 
 /* Waits for `cuda_stream`, then reads and clears the current device's error
- * word: CE_ETARGET if any launch since the last call saw an out-of-range
- * target, CE_ECUDA if the wait itself failed, CE_OK otherwise. */
+ * word: CE_ETIMEOUT if any launch since the last call gave up a bounded wait
+ * (the outputs of that launch, and of the launches that consumed them, are
+ * not valid), else CE_ETARGET if any launch saw an out-of-range target,
+ * CE_ECUDA if the wait itself failed, CE_OK otherwise.
+ *
+ * Bounded waits. The kernels that stream their operands through mbarrier
+ * pipelines (the tensor-core GEMM engine of linear_ce_forward and
+ * linear_ce_backward, and the bulk-copy rings of the long-row kernels) give up
+ * any wait after a time limit (2 s by default; a correct pipeline waits
+ * microseconds): the CTA raises the timeout flag, lets the copies and
+ * tensor-core operations it started complete, frees its tensor memory and
+ * returns, so a broken pipeline ends with an error status instead of a hung
+ * GPU, and the context stays usable. */
 ce_status ce_get_error(void* cuda_stream);
+
+/* Testing hook for the bounded waits; the pages have no counterpart. Sets the
+ * wait limit of the GEMM engine and of the long-row forward's bulk-copy ring
+ * for the launches this process makes afterwards (limit_ns = 0 restores the
+ * default of 2 s). With starve = 1 those launches issue none of their copies,
+ * so every wait for data runs out after the limit: tests use it to check that
+ * a wait that runs out ends the kernel with CE_ETIMEOUT and leaves the
+ * context and the next call correct. starve = 0 is normal operation; any
+ * other value is CE_EINVAL. Not for production use: a starved launch writes
+ * invalid outputs. */
+ce_status ce_testing_set_wait(uint64_t limit_ns, int starve);
 
 /* Static text for a status code. */
 const char* ce_status_string(ce_status s);

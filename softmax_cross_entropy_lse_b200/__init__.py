@@ -22,11 +22,12 @@ LIB_PATH = os.path.join(_HERE, "libce_b200.so")
 CE_F32, CE_BF16, CE_F16 = 0, 1, 2
 CE_I32, CE_I64 = 0, 1
 STATUS = {0: "CE_OK", 1: "CE_EINVAL", 2: "CE_EALIAS", 3: "CE_EWORKSPACE", 4: "CE_ECUDA",
-          5: "CE_ETARGET", 6: "CE_ENOTSUP"}
+          5: "CE_ETARGET", 6: "CE_ENOTSUP", 7: "CE_ETIMEOUT"}
 EXPORTED = ["ce_workspace_size", "ce_forward", "ce_backward", "linear_ce_workspace_size",
             "linear_ce_forward", "linear_ce_backward_workspace_size", "linear_ce_backward",
             "ce_get_error", "ce_status_string", "ce_forward_noalloc", "ce_forward_backward",
-            "ce_soft_forward", "ce_soft_backward", "ce_kl_forward", "ce_kl_backward"]
+            "ce_soft_forward", "ce_soft_backward", "ce_kl_forward", "ce_kl_backward",
+            "ce_testing_set_wait"]
 NOALLOC_SCRATCH_BYTES = 64 << 10
 
 
@@ -91,6 +92,8 @@ def lib() -> ctypes.CDLL:
         L.ce_kl_backward.argtypes = [vp, i64, vp, vp, ctypes.c_int, ce_layout, ce_layout, i64, i64, vp,
                                      vp, vp, vp, vp, ctypes.c_int, ce_layout, vp]
         L.ce_kl_backward.restype = ctypes.c_int
+        L.ce_testing_set_wait.argtypes = [ctypes.c_uint64, ctypes.c_int]
+        L.ce_testing_set_wait.restype = ctypes.c_int
         L.ce_get_error.argtypes = [vp]
         L.ce_get_error.restype = ctypes.c_int
         L.ce_status_string.argtypes = [ctypes.c_int]
@@ -459,6 +462,13 @@ def ce_forward_backward(logits, targets, grad_out, label_smoothing: float = 0.0,
 def get_error(stream=None) -> int:
     """Waits for the stream and returns (and clears) the device error status."""
     return int(lib().ce_get_error(_stream(stream)))
+
+
+def testing_set_wait(limit_ns: int = 0, starve: bool = False) -> None:
+    """Testing hook of the bounded pipeline waits (ce_testing_set_wait): the
+    wait limit for later launches (0 = the default) and whether they issue
+    no copies, so that their waits run out. Not for production use."""
+    _check(lib().ce_testing_set_wait(int(limit_ns), 1 if starve else 0), "ce_testing_set_wait")
 
 
 # -- fused-linear cross-entropy ----------------------------------------------------------

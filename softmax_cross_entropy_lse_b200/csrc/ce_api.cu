@@ -1,11 +1,14 @@
 // C ABI of the fused softmax cross-entropy library: argument validation,
 // workspace sizing, kernel planning and launches. No allocation, no
 // synchronisation on the hot path.
+#include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "ce_b200.h"
 #include "ce_launch.h"
 #include "ce_linear.h"
+#include "ce_sm100.cuh"
 
 namespace ceb {
 
@@ -47,6 +50,36 @@ int device_sms(int num_sms) {
         g_num_sms[dev] = n;
     }
     return g_num_sms[dev];
+}
+
+// Settings of the testing hook ce_testing_set_wait.
+static std::atomic<unsigned long long> g_wait_limit_ns{0};  // 0: the default
+static std::atomic<int> g_wait_starve{0};
+
+WaitPolicy wait_policy() {
+    const unsigned long long ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+    return WaitPolicy{ns ? ns : sm100::kWaitTimeoutNs, g_wait_starve.load(std::memory_order_relaxed)};
+}
+
+// (kernel, device) pairs whose shared-memory limit has been raised, with the
+// bytes it was raised to.
+struct SmemLimit {
+    const void* kernel;
+    int device, bytes;
+};
+static std::vector<SmemLimit> g_smem_limits;
+
+cudaError_t ensure_smem_limit(const void* kernel, int bytes) {
+    const int dev = current_device();
+    if (dev < 0) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    for (const SmemLimit& l : g_smem_limits)
+        if (l.kernel == kernel && l.device == dev && l.bytes >= bytes) return cudaSuccess;
+    const cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    g_smem_limits.push_back(SmemLimit{kernel, dev, bytes});
+    return cudaSuccess;
 }
 
 int elem_size(int dt) { return dt == CE_F32 ? 4 : 2; }
@@ -320,6 +353,9 @@ ce_status ce_forward(const void* logits, ce_dtype dt, ce_layout lg, int64_t N, i
     a.vec_per_split = plan.vec_per_split;
     a.lz = L;
     a.ly = T;
+    const WaitPolicy wp = wait_policy();
+    a.wait_ns = wp.limit_ns;
+    a.starve = wp.starve;
     cudaError_t e = launch_forward(plan, a, (int)dt, static_cast<cudaStream_t>(cuda_stream));
     return e == cudaSuccess ? CE_OK : CE_ECUDA;
 }
@@ -725,6 +761,7 @@ ce_status ce_forward_backward(const void* logits, ce_dtype dt, ce_layout lg, int
     a.f.splits = 1;
     a.f.lz = L;
     a.f.ly = T;
+    a.f.wait_ns = wait_policy().limit_ns;
     a.g = grad_out;
     a.g_stride = grad_stride;
     a.dz = dlogits;
@@ -742,8 +779,16 @@ ce_status ce_get_error(void* cuda_stream) {
     if (w) {
         const unsigned int zero = 0;
         if (cudaMemcpyToSymbol(g_ce_error_word, &zero, sizeof(zero)) != cudaSuccess) return CE_ECUDA;
-        return CE_ETARGET;
+        // a wait that ran out invalidates whole launches: it outranks a bad target
+        return (w & kErrTimeout) ? CE_ETIMEOUT : CE_ETARGET;
     }
+    return CE_OK;
+}
+
+ce_status ce_testing_set_wait(uint64_t limit_ns, int starve) {
+    if (starve != 0 && starve != 1) return CE_EINVAL;
+    g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+    g_wait_starve.store(starve, std::memory_order_relaxed);
     return CE_OK;
 }
 
@@ -756,6 +801,7 @@ const char* ce_status_string(ce_status s) {
         case CE_ECUDA: return "CUDA runtime error";
         case CE_ETARGET: return "a target outside [0, V) that is not ignore_index";
         case CE_ENOTSUP: return "configuration not supported";
+        case CE_ETIMEOUT: return "a kernel gave up a bounded wait; the outputs of that launch are not valid";
     }
     return "unknown status";
 }

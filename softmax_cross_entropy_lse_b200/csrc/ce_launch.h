@@ -7,6 +7,23 @@
 
 namespace ceb {
 
+// Bit of the device error word raised by a kernel that gave up a bounded
+// pipeline wait (bit 0 flags an out-of-range target).
+constexpr unsigned kErrTimeout = 2u;
+
+// Time limit of the bounded pipeline waits and the copy-starving switch of
+// the testing hook ce_testing_set_wait (defaults: 2 s, off). Read at launch
+// time and passed to the kernels that wait on mbarriers for their copies.
+struct WaitPolicy {
+    unsigned long long limit_ns;
+    int starve;  // 1: producers issue no copies, so every wait for data runs out
+};
+WaitPolicy wait_policy();
+
+// Raises the dynamic shared-memory limit of `kernel` to `bytes` on the
+// current device, once per (kernel, device); safe from several threads.
+cudaError_t ensure_smem_limit(const void* kernel, int bytes);
+
 // Two-level row addressing: row r starts at (r / inner) * s_outer +
 // (r % inner) * s_inner elements, column j a further j * s_col on.
 struct Layout {
@@ -31,6 +48,8 @@ struct FwdArgs {
     int vec_is_scalar;
     int64_t vec_per_split;  // in units of the kernel's vector width
     Layout lz, ly;
+    unsigned long long wait_ns;  // limit of the bulk-copy ring's waits
+    int starve;                  // testing: the ring issues no copies
 };
 
 struct FwdPlan {

@@ -43,7 +43,6 @@ constexpr int kGemmThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilo
 constexpr uint32_t kTmemCols = 2 * kBN;
 constexpr size_t kGemmSmem = 1024 + (size_t)kStages * kStageBytes + 256;
 constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN);
-constexpr unsigned kErrTimeout = 2u;
 
 enum EpiKind { kEpiCeFwd = 0, kEpiCeGrad = 1, kEpiStore = 2, kEpiAccum = 3 };
 
@@ -55,6 +54,8 @@ struct GemmArgs {
     int64_t units;             // n_mb * n_units_n
     int kA0, kB0;              // K origin of A and B in their tensor maps
     unsigned int* err;
+    unsigned long long wait_ns;  // limit of every pipeline wait
+    int starve;                  // testing: the producer issues no copies
     // cross-entropy epilogues
     const void* y;
     int tdt;
@@ -202,17 +203,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int nb1 = min(a.n_nb, nb0 + a.tiles_per_unit);
                 for (int nb = nb0; nb < nb1 && ok; ++nb) {
                     for (int kb = 0; kb < a.nkb; ++kb) {
-                        if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag)) {
+                        if (!mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, a.wait_ns)) {
                             ok = false;
                             break;
                         }
-                        mbar_expect_tx(full_bar(s), kStageBytes);
-                        tma_load_2d(smem_u32(sA + s * kABytes), &tmA, full_bar(s),
-                                    a.kA0 + kb * kBK, mb * kBM);
-                        tma_load_2d(smem_u32(sB + s * kBBytes), &tmB, full_bar(s),
-                                    a.kB0 + kb * kBK, nb * kBN);
-                        issued_mask |= 1u << s;
-                        last_ph = (last_ph & ~(1u << s)) | (ph << s);
+                        // (a starved launch, a testing mode, issues no copies:
+                        // the MMA thread's wait for this stage runs out)
+                        if (!a.starve) {
+                            mbar_expect_tx(full_bar(s), kStageBytes);
+                            tma_load_2d(smem_u32(sA + s * kABytes), &tmA, full_bar(s),
+                                        a.kA0 + kb * kBK, mb * kBM);
+                            tma_load_2d(smem_u32(sB + s * kBBytes), &tmB, full_bar(s),
+                                        a.kB0 + kb * kBK, nb * kBN);
+                            issued_mask |= 1u << s;
+                            last_ph = (last_ph & ~(1u << s)) | (ph << s);
+                        }
                         if (++s == kStages) {
                             s = 0;
                             ph ^= 1u;
@@ -240,14 +245,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int nb1 = min(a.n_nb, nb0 + a.tiles_per_unit);
                 for (int nb = nb0; nb < nb1 && ok; ++nb, ++it) {
                     const uint32_t acc = it & 1u;
-                    if (!mbar_wait(tempty_bar(acc), ((it >> 1) & 1u) ^ 1u, abort_flag)) {
+                    if (!mbar_wait(tempty_bar(acc), ((it >> 1) & 1u) ^ 1u, abort_flag, a.wait_ns)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t d = tmem_base + acc * kBN;
                     for (int kb = 0; kb < a.nkb; ++kb) {
-                        if (!mbar_wait(full_bar(s), ph, abort_flag)) {
+                        if (!mbar_wait(full_bar(s), ph, abort_flag, a.wait_ns)) {
                             ok = false;
                             break;
                         }
@@ -311,7 +316,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
             for (int nb = nb0; nb < nb1; ++nb, ++it) {
                 const uint32_t acc = it & 1u;
-                if (!mbar_wait(tfull_bar(acc), (it >> 1) & 1u, abort_flag)) {
+                if (!mbar_wait(tfull_bar(acc), (it >> 1) & 1u, abort_flag, a.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -497,13 +502,11 @@ static bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t c
 template <int EPI>
 static cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmArgs a, int sms,
                                cudaStream_t s) {
-    static bool attr_set[4] = {false, false, false, false};
-    if (!attr_set[EPI]) {
-        cudaError_t e = cudaFuncSetAttribute(k_gemm<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kGemmSmem);
-        if (e != cudaSuccess) return e;
-        attr_set[EPI] = true;
-    }
+    cudaError_t e = ensure_smem_limit((const void*)k_gemm<EPI>, (int)kGemmSmem);
+    if (e != cudaSuccess) return e;
+    const WaitPolicy wp = wait_policy();
+    a.wait_ns = wp.limit_ns;
+    a.starve = wp.starve;
     a.n_mb = (a.M + kBM - 1) / kBM;
     a.n_nb = (a.Nn + kBN - 1) / kBN;
     a.nkb = (a.K + kBK - 1) / kBK;

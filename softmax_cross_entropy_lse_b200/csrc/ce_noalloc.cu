@@ -1,20 +1,23 @@
 // ce_forward_noalloc: the row cross-entropy forward for callers that cannot
 // allocate device memory.
 //
-// Some callers cannot call cudaMalloc or hand over a workspace: code that runs
-// while a stream is being captured into a graph (allocation is not a stream
-// operation and is refused there), plugin hosts that own every byte of the
-// device through their own pool, or C callers with no allocator at hand. The
-// split-vocabulary forward needs scratch memory for its per-row partial
-// states; this entry point takes that scratch from a fixed array in device
-// memory that belongs to the library instead.
+// Some callers cannot call cudaMalloc or hand over a workspace: plugins that
+// run inside a host application which owns every byte of the device through
+// its own pool (a raw allocation would bypass its accounting or exceed its
+// budget), loops with a fixed memory budget set at start-up that must not run
+// out of memory halfway, and C callers with no allocator at hand (cudaMalloc
+// may also synchronise the device, which a latency-bound caller cannot
+// afford). The split-vocabulary forward needs scratch memory for its per-row
+// partial states; this entry point takes that scratch from a fixed array in
+// device memory that belongs to the library instead.
 //
 // The array is a file-scope __device__ variable of kScratchBytes bytes. Every
 // device that loads the library holds one copy until the process exits.
 // Host code cannot use the array's name as a device address (on the host it
 // names a stand-in object), so the device address is looked up once per
 // device with cudaGetSymbolAddress, with that device current, on the first
-// call made on it, and cached.
+// call made on it, and cached; that first call on a device should come before
+// any stream capture begins.
 #include <mutex>
 
 #include "ce_b200.h"

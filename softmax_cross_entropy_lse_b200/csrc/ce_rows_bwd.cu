@@ -509,7 +509,7 @@ __global__ void __launch_bounds__(kBRingWarps * 32, 2) k_bwd_ring(BwdArgs a) {
     }
     if (dead || abort_flag) {
         if (lane == 0) {
-            atomicOr(a.err, 2u);
+            atomicOr(a.err, kErrTimeout);
             volatile int never = 0;
             for (int64_t e = waited; e < issued; ++e)
                 mbar_wait(smem_u32(&full_bar[wid][e % kBRingStages]),
@@ -520,14 +520,8 @@ __global__ void __launch_bounds__(kBRingWarps * 32, 2) k_bwd_ring(BwdArgs a) {
 
 template <typename TI, typename TO>
 static cudaError_t launch_bwd_ring(const BwdPlan& p, const BwdArgs& a, cudaStream_t s) {
-    static bool attr = false;  // per process; the library targets one device per process
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(k_bwd_ring<TI, TO>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kBRingSmem);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    cudaError_t e = ensure_smem_limit((const void*)k_bwd_ring<TI, TO>, (int)kBRingSmem);
+    if (e != cudaSuccess) return e;
     k_bwd_ring<TI, TO><<<p.grid, kBRingWarps * 32, kBRingSmem, s>>>(a);
     return cudaGetLastError();
 }

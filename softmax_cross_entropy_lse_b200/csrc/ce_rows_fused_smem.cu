@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
     }
 
     if (dead || abort_flag) {
-        if (lane == 0) atomicOr(a.err, 2u);
+        if (lane == 0) atomicOr(a.err, kErrTimeout);
         // let every copy this warp started land before the CTA exits
         volatile int never = 0;
         for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps)
@@ -332,12 +332,9 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
 template <typename TI, typename TO, int CL, bool ARGMAX, bool WITH_T>
 static cudaError_t launch_smem_k(const SmemRowPlan& sp, const FusedArgs& a, cudaStream_t s) {
     auto kern = k_fwdbwd_smem<TI, TO, CL, ARGMAX, WITH_T>;
-    static std::atomic<int> attr{0};
-    if (!attr.load(std::memory_order_relaxed)) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kSmMaxChunks * 2048);
+    {
+        cudaError_t e = ensure_smem_limit((const void*)kern, kSmMaxChunks * 2048);
         if (e != cudaSuccess) return e;
-        attr.store(1, std::memory_order_relaxed);
     }
     const size_t smem = (size_t)sp.nch * 2048;
     cudaLaunchConfig_t cfg = {};

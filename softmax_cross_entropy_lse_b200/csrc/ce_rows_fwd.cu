@@ -420,13 +420,16 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
     // 32-bit counters: stage = count % kRingStages and parity = (count /
     // kRingStages) % 2 stay exact across wraparound (powers of two divide 2^32)
     uint32_t issued = 0;
+    // (a starved launch, a testing mode, issues no copies: its waits run out)
     for (int q = 0; q < kRingStages && iss.valid(units); ++q) {
-        if (lane == 0) {
-            const uint32_t bar = smem_u32(&full_bar[wid][q]);
-            mbar_expect_tx(bar, iss.bytes());
-            bulk_load(smem_u32(ring + q * kRingVecs * 16), iss.src(), iss.bytes(), bar);
+        if (!a.starve) {
+            if (lane == 0) {
+                const uint32_t bar = smem_u32(&full_bar[wid][q]);
+                mbar_expect_tx(bar, iss.bytes());
+                bulk_load(smem_u32(ring + q * kRingVecs * 16), iss.src(), iss.bytes(), bar);
+            }
+            ++issued;
         }
-        ++issued;
         iss.next(a, units, nvec, wid);
     }
 
@@ -453,7 +456,7 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
             const int stage = (int)(consumed & (kRingStages - 1));
             const uint32_t bar = smem_u32(&full_bar[wid][stage]);
             if (!dead) {
-                if (mbar_wait(bar, (consumed / kRingStages) & 1u, &abort_flag))
+                if (mbar_wait(bar, (consumed / kRingStages) & 1u, &abort_flag, a.wait_ns))
                     ++waited;
                 else
                     dead = true;
@@ -505,7 +508,7 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
             // the buffer is read: hand it back to the copy engine
             fence_proxy_async_smem();
             __syncwarp();
-            if (iss.valid(units) && !dead) {
+            if (iss.valid(units) && !dead && !a.starve) {
                 if (lane == 0) {
                     mbar_expect_tx(bar, iss.bytes());
                     bulk_load(smem_u32(ring + stage * kRingVecs * 16), iss.src(), iss.bytes(), bar);
@@ -551,7 +554,7 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
         }
     }
     if (dead || abort_flag) {
-        if (lane == 0) atomicOr(a.err, 2u);
+        if (lane == 0) atomicOr(a.err, kErrTimeout);
         // let every copy this warp started land before the CTA exits
         if (lane == 0) {
             volatile int never = 0;
@@ -627,14 +630,8 @@ static cudaError_t launch_packed(const FwdArgs& a, int G, int U, int grid, cudaS
 
 template <typename T, bool ARGMAX, bool WITH_T>
 static cudaError_t launch_ring(const FwdPlan& p, const FwdArgs& a, cudaStream_t s) {
-    static bool attr = false;  // per process; the library targets one device per process
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(k_fwd_ring<T, ARGMAX, WITH_T>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)kRingSmem);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    cudaError_t e = ensure_smem_limit((const void*)k_fwd_ring<T, ARGMAX, WITH_T>, (int)kRingSmem);
+    if (e != cudaSuccess) return e;
     k_fwd_ring<T, ARGMAX, WITH_T><<<p.grid, kRingWarps * 32, kRingSmem, s>>>(a);
     return cudaGetLastError();
 }
@@ -645,14 +642,9 @@ static cudaError_t launch_pipe(const FwdPlan& p, const FwdArgs& a, cudaStream_t 
     constexpr size_t smem = (size_t)2 * kPipeWarps * U * 32 * 16;  // 64 KB
 #define CEB_PIPE(GG)                                                                            \
     if (p.G == GG) {                                                                            \
-        static bool attr = false;                                                               \
-        if (!attr) {                                                                            \
-            cudaError_t e = cudaFuncSetAttribute(k_fwd_packed_pipe<T, VEC, GG, U, false, 3>,     \
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,   \
-                                                 (int)smem);                                    \
-            if (e != cudaSuccess) return e;                                                     \
-            attr = true;                                                                        \
-        }                                                                                       \
+        cudaError_t e =                                                                         \
+            ensure_smem_limit((const void*)k_fwd_packed_pipe<T, VEC, GG, U, false, 3>, (int)smem); \
+        if (e != cudaSuccess) return e;                                                         \
         k_fwd_packed_pipe<T, VEC, GG, U, false, 3><<<p.grid, kPipeWarps * 32, smem, s>>>(a);    \
         return cudaGetLastError();                                                              \
     }

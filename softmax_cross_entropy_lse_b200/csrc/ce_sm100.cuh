@@ -24,7 +24,8 @@
 namespace ceb {
 namespace sm100 {
 
-// Every wait gives up after this long (a correct pipeline waits microseconds).
+// Every wait gives up after this long by default (a correct pipeline waits
+// microseconds); kernels that take a limit as an argument use theirs.
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -88,15 +89,17 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t par
 constexpr uint32_t kSuspendHintNs = 20000;
 
 // Waits for the phase of parity `parity` to complete. Returns false (and
-// raises *abort) when the time limit passes or another role already aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+// raises *abort) when `limit_ns` nanoseconds pass or another role already
+// aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          unsigned long long limit_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) return true;
         if ((i & 15u) == 0) {
             if (*abort) return false;
-            if (globaltimer() - t0 > kWaitTimeoutNs) {
+            if (globaltimer() - t0 > limit_ns) {
                 *abort = 1;
                 return false;
             }

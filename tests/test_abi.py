@@ -40,9 +40,19 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_status_strings(L):
-    for s in range(7):
+    for s in range(8):
         assert L.ce_status_string(s)
     assert L.ce_status_string(99) == b"unknown status"
+    assert b"bounded wait" in L.ce_status_string(7)
+
+
+def test_wait_hook_validates_and_resets(L):
+    """The testing hook of the bounded waits takes starve 0 or 1 only; the
+    settings are host state, so this needs no GPU."""
+    assert L.ce_testing_set_wait(0, 2) == 1
+    assert L.ce_testing_set_wait(0, -1) == 1
+    assert L.ce_testing_set_wait(10_000_000, 1) == 0
+    assert L.ce_testing_set_wait(0, 0) == 0
 
 
 def lay(N, ld, s_col=1):

@@ -1,6 +1,7 @@
 """ce_forward_noalloc: the forward for callers that cannot allocate device
-memory (code running during CUDA graph capture, hosts that own all device
-memory through their own pool, C callers without an allocator).
+memory (plugins inside a host application that owns all device memory
+through its own pool, loops with a memory budget fixed at start-up, C callers
+without an allocator; cudaMalloc may also synchronise the device).
 
 It runs the vocabulary-split forward with its scratch in a library-owned
 static device array instead of a caller workspace. These tests call it
