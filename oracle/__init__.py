@@ -51,6 +51,8 @@ class Oracle:
                                                  _i64p, ctypes.c_double, _i64, _f64p, _f64p]
         L.orc_linear_ce_dh_rows.argtypes = [_f32p, _f32p, _i64, _i64, _i64p, _i64, _i64p,
                                             _f64p, ctypes.c_double, _i64, _f64p]
+        L.orc_linear_ce_dw_rows.argtypes = [_f32p, _f32p, _i64, _i64, _i64, _i64p, _i64, _i64p,
+                                            _f64p, _f64p, ctypes.c_double, _i64, _f64p]
         L.orc_linear_ce_backward.argtypes = [_f32p, _f32p, _i64, _i64, _i64, _i64p, _f64p,
                                              ctypes.c_double, _i64, _f64p, _f64p, _f64p]
         L.orc_ce_soft_forward.argtypes = [_f64p, _f64p, _i64, _i64, ctypes.c_double, _f64p, _f64p]
@@ -174,6 +176,47 @@ class Oracle:
                                        self._p(g, _f64p), float(eps), int(ignore_index),
                                        self._p(dH, _f64p))
         return dH
+
+    def linear_ce_dw_rows(self, H, W, y, g, cols, lse, eps: float = 0.0,
+                          ignore_index: int = -100):
+        """Rows of dW = G^T H for the listed vocabulary indices, float64
+        (len(cols), D); lse (N,) is every row's log-sum-exp (float64)."""
+        H = np.ascontiguousarray(H, dtype=np.float32)
+        W = np.ascontiguousarray(W, dtype=np.float32)
+        y = np.ascontiguousarray(y, dtype=np.int64)
+        N, D = H.shape
+        V = W.shape[0]
+        g = np.ascontiguousarray(np.broadcast_to(np.asarray(g, np.float64), (N,)))
+        lse = np.ascontiguousarray(lse, dtype=np.float64)
+        assert lse.shape == (N,)
+        cols = np.ascontiguousarray(cols, dtype=np.int64)
+        dW = np.empty((len(cols), D), np.float64)
+        self.lib.orc_linear_ce_dw_rows(self._p(H, _f32p), self._p(W, _f32p), N, V, D,
+                                       self._p(cols, _i64p), len(cols), self._p(y, _i64p),
+                                       self._p(g, _f64p), self._p(lse, _f64p), float(eps),
+                                       int(ignore_index), self._p(dW, _f64p))
+        return dW
+
+    @staticmethod
+    def linear_lse_all(H, W, chunk: int = 8192):
+        """lse_i = m_i + log sum_j exp(Z_ij - m_i) of every row of Z = H W^T
+        in float64, for problems too large for the row-by-row C loop (every
+        row of the fused-linear workload). Z is formed one vocabulary chunk at
+        a time by numpy's float64 matrix product (a library primitive); a
+        first pass over the chunks takes the row maxima m_i, a second the sums
+        of exp(Z_ij - m_i), chunk after chunk in vocabulary order."""
+        Hd = np.asarray(H, dtype=np.float64)
+        N = Hd.shape[0]
+        V = W.shape[0]
+        m = np.full(N, -np.inf)
+        for v0 in range(0, V, chunk):
+            Z = Hd @ np.asarray(W[v0:v0 + chunk], dtype=np.float64).T
+            np.maximum(m, Z.max(axis=1), out=m)
+        s = np.zeros(N)
+        for v0 in range(0, V, chunk):
+            Z = Hd @ np.asarray(W[v0:v0 + chunk], dtype=np.float64).T
+            s += np.exp(Z - m[:, None]).sum(axis=1)
+        return m + np.log(s)
 
     def linear_ce_backward(self, H, W, y, g, eps: float = 0.0, ignore_index: int = -100):
         """dH (N, D) and dW (V, D) in float64 for a small problem; also G (N, V)."""

@@ -212,6 +212,46 @@ void orc_linear_ce_dh_rows(const float* H, const float* W, int64_t V,
     }
 }
 
+/* Fused-linear backward for selected vocabulary entries: the rows of
+ * dW = G^T H (the chain rule through Z = H W^T, Ineshin section 1) for the
+ * listed vocabulary indices. Column v of the logit gradient needs only
+ * column v of Z, z_iv = H_i . W_v (double, d in order), and the log-sum-exp
+ * lse_i of every row (an input: the forward over the full rows), so
+ *   G_iv = g_i (exp(z_iv - lse_i) - (1-eps)[v = y_i] - eps/V)
+ * (zero for ignore_index rows, NaN for a target outside [0, V)), and
+ *   dW_v = sum_i G_iv H_i, i in order.
+ * dW: ncols*D doubles, indexed by position in cols. */
+void orc_linear_ce_dw_rows(const float* H, const float* W, int64_t N, int64_t V,
+                           int64_t D, const int64_t* cols, int64_t ncols,
+                           const int64_t* y, const double* g, const double* lse,
+                           double eps, int64_t ignore_index, double* dW)
+{
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t k = 0; k < ncols; ++k) {
+        const int64_t v = cols[k];
+        const float* w = W + v * D;
+        double* out = dW + k * D;
+        for (int64_t d = 0; d < D; ++d) out[d] = 0.0;
+        for (int64_t i = 0; i < N; ++i) {
+            double giv;
+            if (y[i] == ignore_index) {
+                giv = 0.0;
+            } else if (y[i] < 0 || y[i] >= V) {
+                giv = NAN;
+            } else {
+                const float* h = H + i * D;
+                double z = 0.0;
+                for (int64_t d = 0; d < D; ++d) z += (double)h[d] * (double)w[d];
+                const double onehot = (v == y[i]) ? 1.0 : 0.0;
+                giv = g[i] * (exp(z - lse[i]) - (1.0 - eps) * onehot - eps / (double)V);
+            }
+            if (giv == 0.0) continue;
+            const float* h = H + i * D;
+            for (int64_t d = 0; d < D; ++d) out[d] += giv * (double)h[d];
+        }
+    }
+}
+
 /* Full fused-linear backward for small problems: G = dloss/dZ (N x V double,
  * caller-provided scratch), dH = G W (N x D), dW = G^T H (V x D). Sums over
  * the contracted index run in order. */

@@ -286,6 +286,13 @@ def pin_linear_vs_numpy(orc):
         rows = np.array([0, 4, 23, 9])
         dHr = orc.linear_ce_dh_rows(H, W, y, g, rows, eps=eps)
         np.testing.assert_allclose(dHr, dH[rows], rtol=1e-12, atol=1e-15)
+        # dW rows from single columns of Z, given numpy's lse of every row
+        cols = np.array([0, int(y[0]), 36, 17, int(y[5])])
+        dWr = orc.linear_ce_dw_rows(H, W, y, g, cols, lsez, eps=eps)
+        np.testing.assert_allclose(dWr, (G.T @ H.astype(np.float64))[cols], rtol=1e-11,
+                                   atol=1e-14)
+        # the chunked float64 lse of every row: numpy's lse over the whole Z
+        np.testing.assert_allclose(orc.linear_lse_all(H, W, chunk=8), lsez, rtol=1e-14)
         lr, _ = orc.linear_ce_forward_rows(H, W, y, rows=rows, eps=eps)
         np.testing.assert_allclose(lr, lf[rows], rtol=1e-15)
 
@@ -316,6 +323,11 @@ def pin_linear_finite_differences(orc):
                 fm = f(Am, W) if which == 0 else f(H, Am)
                 fd[idx] = (fp - fm) / (2 * h)
             np.testing.assert_allclose(dA, fd, rtol=0, atol=5e-7)
+        # the dW rows of single Z columns against the same differences
+        _, lse = orc.linear_ce_forward_rows(H, W, y, eps=eps)
+        cols = np.arange(V)
+        np.testing.assert_allclose(orc.linear_ce_dw_rows(H, W, y, g, cols, lse, eps=eps), dW,
+                                   rtol=0, atol=1e-12)
 
 
 # ---- probability (soft) targets ---------------------------------------------------

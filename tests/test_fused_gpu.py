@@ -47,7 +47,7 @@ def check_oracle(orc, r, dz, z64, y, g, eps, ignore, in_dt, out_dt):
     assert_close(f32(r.lse), lse, rt, at, "lse")
     np.testing.assert_array_equal(r.argmax.cpu().numpy(), am)
     ref = orc.ce_backward(z64, y, g, eps, ignore)
-    assert_grad_close(f32(dz).reshape(z64.shape), ref, in_dt, out_dt)
+    assert_grad_close(f32(dz).reshape(z64.shape), ref, in_dt, out_dt, g=g)
 
 
 def test_c2_fused_matches_separate(orc):
@@ -169,7 +169,7 @@ def test_smem_rows_vs_oracle(orc, V, N, dt):
         if am:
             np.testing.assert_array_equal(rf.argmax.cpu().numpy(), amx)
         ref = orc.ce_backward(z32.astype(np.float64), y, gv.astype(np.float64), eps)
-        assert_grad_close(f32(dzf), ref, dt, dt)
+        assert_grad_close(f32(dzf), ref, dt, dt, g=gv)
         # the same lse as the separate forward, up to the order of the sum
         rs = ce.ce_forward(zt, yt, eps)
         assert_close(f32(rf.lse), f32(rs.lse).astype(np.float64), 2e-6, 0.0, "lse vs ce_forward")
@@ -276,7 +276,7 @@ def test_tiny_rows_fused(orc, V, dt, out):
         if am:
             np.testing.assert_array_equal(rf.argmax.cpu().numpy(), amx)
         ref = orc.ce_backward(z32.astype(np.float64), y, gv.astype(np.float64), eps)
-        assert_grad_close(f32(dzf), ref, dt, out)
+        assert_grad_close(f32(dzf), ref, dt, out, g=gv)
 
 
 def test_tiny_rows_fused_in_place_view(orc):

@@ -71,6 +71,13 @@ MUTANTS = [
     ("dH contracts with H", "acc += G[i * V + j] * (double)W[j * D + d];\n            dH",
      "acc += G[i * V + j] * (double)H[i * D + d];\n            dH"),
     ("dh rows sign", "out[d] += gij * (double)w[d];", "out[d] -= gij * (double)w[d];"),
+    ("dw rows contract with W", "out[d] += giv * (double)h[d];", "out[d] += giv * (double)w[d];"),
+    ("dw rows drop eps/V", "- (1.0 - eps) * onehot - eps / (double)V);",
+     "- (1.0 - eps) * onehot);"),
+    ("dw rows one-hot on the row index", "const double onehot = (v == y[i]) ? 1.0 : 0.0;",
+     "const double onehot = (i == y[i]) ? 1.0 : 0.0;"),
+    ("dw rows keep ignored rows", "if (y[i] == ignore_index) {\n                giv = 0.0;",
+     "if (0) {\n                giv = 0.0;"),
     ("soft lse drops m", "*lse = m + L;", "*lse = L;"),
     ("soft exp unshifted", "s += exp(z[j] - m);\n    const double L", "s += exp(z[j]);\n    const double L"),
     ("soft loss sign", "l += tj * (L - (z[j] - m));", "l += tj * (L + (z[j] - m));"),

@@ -44,7 +44,7 @@ def check(orc, r, dz, z32, t32, g, eps, dt, od):
     assert_close(f32(r.lse), lse, rt, at, "lse")
     np.testing.assert_allclose(f32(r.target_sum), t32.astype(np.float64).sum(1), rtol=1e-5, atol=1e-6)
     ref = orc.ce_soft_backward(z32.astype(np.float64), t32.astype(np.float64), g, eps)
-    assert_grad_close(f32(dz).reshape(ref.shape), ref, dt, od)
+    assert_grad_close(f32(dz).reshape(ref.shape), ref, dt, od, g=g)
 
 
 @pytest.mark.parametrize("V", [1, 3, 8, 100, 1000, 1023, 4099, 32000])
