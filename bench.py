@@ -53,6 +53,27 @@ ROW_WORKLOADS = {
 }
 
 
+# Data-sheet peaks, reported beside the measured ones: HBM3e 8 TB/s and
+# 2.25 PFLOP/s dense bf16 for one B200.
+SPEC_HBM_GBS = 8000.0
+SPEC_BF16_TFLOPS = 2250.0
+
+
+def roofline(bound, kernel, achieved, peak, peak_src, traffic, algorithmic=None):
+    """The roofline object of a JSON line: the fraction of the measured peak
+    (the copy or GEMM rate measured on this machine's B200s) and, beside it, the
+    fraction of the data-sheet peak."""
+    spec = SPEC_HBM_GBS if bound == "hbm" else SPEC_BF16_TFLOPS
+    r = {"bound": bound, "kernel": kernel, "achieved": round(achieved, 2), "peak": peak,
+         "unit": "GB/s" if bound == "hbm" else "TFLOP/s", "frac": round(achieved / peak, 4),
+         "traffic": traffic, "peak_source": peak_src, "spec_peak": spec,
+         "frac_of_spec": round(achieved / spec, 4)}
+    if algorithmic is not None:
+        r["algorithmic_bytes_per_launch" if bound == "hbm" else "algorithmic_flop_per_launch"] = \
+            algorithmic
+    return r
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -374,10 +395,8 @@ def bench_rows(args, rk):
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 2),
-                     "peak": peak_hbm, "unit": "GB/s", "frac": round(achieved / peak_hbm, 4),
-                     "traffic": recorded_traffic(args.workload, dom),
-                     "peak_source": peak_src, "algorithmic_bytes_per_launch": dom_bytes},
+        "roofline": roofline("hbm", dom, achieved, peak_hbm, peak_src,
+                             recorded_traffic(args.workload, dom), dom_bytes),
     }
     if fused_ms is not None:
         fused_bytes = 2 * N * V * esz + 16 * N
@@ -389,6 +408,11 @@ def bench_rows(args, rk):
     if args.workload in PAGE_FWD_BWD_MS:
         page_gbs = step_bytes / (PAGE_FWD_BWD_MS[args.workload] * 1e-3) / 1e9
         out["vs_baseline"] = round(value / page_gbs, 2)
+        out["vs_apple_m5pro_mlx"] = out["vs_baseline"]
+        out["vs_baseline_basis"] = (
+            f"value / the pages' Apple M5 Pro MLX rate for this shape ({page_gbs:.1f} GB/s from "
+            f"{PAGE_FWD_BWD_MS[args.workload]} ms forward + backward, MLX PR #4776 Benchmarks, "
+            "fix column): another machine's number, context only")
     clocks = clk.summary()
     if clocks:
         out["clocks"] = clocks
@@ -493,10 +517,8 @@ def bench_soft(args, rk):
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": 2 * N * V * 2, "d2h_bytes_per_step": 4 * N},
         "gpu_launches": 2 * args.steps,
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 2), "peak": peak_hbm,
-                     "unit": "GB/s", "frac": round(achieved / peak_hbm, 4),
-                     "traffic": recorded_traffic("soft", dom),
-                     "peak_source": peak_src, "algorithmic_bytes_per_launch": dom_bytes},
+        "roofline": roofline("hbm", dom, achieved, peak_hbm, peak_src,
+                             recorded_traffic("soft", dom), dom_bytes),
     }
     clocks = clk.summary()
     if clocks:
@@ -597,10 +619,8 @@ def bench_kl(args, rk):
         "e2e": {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": 2 * N * V * 4, "d2h_bytes_per_step": 4 * N},
         "gpu_launches": 2 * args.steps,
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 2), "peak": peak_hbm,
-                     "unit": "GB/s", "frac": round(achieved / peak_hbm, 4),
-                     "traffic": recorded_traffic("kl", dom),
-                     "peak_source": peak_src, "algorithmic_bytes_per_launch": dom_bytes},
+        "roofline": roofline("hbm", dom, achieved, peak_hbm, peak_src,
+                             recorded_traffic("kl", dom), dom_bytes),
     }
     clocks = clk.summary()
     if clocks:
@@ -701,9 +721,8 @@ def bench_linear(args, rk):
         "e2e": {"value": round(world * step_flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": (N * D + V * D) * 2 + 4 * N, "d2h_bytes_per_step": 4 * N},
         "gpu_launches": (2 + 1 + 4 * ((V + 8191) // 8192)) * args.steps,
-        "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 2),
-                     "peak": peak_sust, "unit": "TFLOP/s", "frac": round(achieved / peak_sust, 4),
-                     "traffic": recorded_traffic("c5", dom), "peak_source": src + " (sustained)"},
+        "roofline": roofline("tensor", dom, achieved, peak_sust, src + " (sustained)",
+                             recorded_traffic("c5", dom), dom_flop),
     }
     clocks = clk.summary()
     if clocks:
@@ -899,12 +918,47 @@ def run_reference(args):
     return 0
 
 
+EXTRA_WORKLOADS = ["c1", "c3a", "c3b", "c4a", "c4b", "c5", "soft", "kl"]
+SUMMARY_KEYS = ("value", "unit", "ms_per_step", "steps", "dtype", "rows_per_s", "fwd_GBs",
+                "fwd_rows_per_s", "bwd_GBs", "fwd_tflops", "fwd_ms", "bwd_ms", "workspace_bytes",
+                "vs_baseline", "vs_baseline_basis", "gpu_launches", "roofline", "fused", "clocks",
+                "e2e", "config", "dense_vs_fused")
+
+
+def run_workload(args, rk, name):
+    if name == "c5":
+        return bench_linear(args, rk)
+    if name == "soft":
+        return bench_soft(args, rk)
+    if name == "kl":
+        return bench_kl(args, rk)
+    args.workload = name
+    return bench_rows(args, rk)
+
+
+def workload_summary(out: dict) -> dict:
+    """The parts of a workload's JSON line kept under the headline's 'workloads'."""
+    return {k: out[k] for k in SUMMARY_KEYS if k in out}
+
+
+def release_device_memory() -> None:
+    import gc
+    import torch
+    gc.collect()
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="c2", choices=sorted(ROW_WORKLOADS) + ["c5", "soft", "kl"])
+    ap.add_argument("--also", default=None,
+                    help="comma-separated workloads measured after the headline one and reported "
+                         "under 'workloads' (default: every other workload when the headline is "
+                         "c2, none otherwise; 'none' for none)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rows", type=int, default=0,
@@ -921,18 +975,27 @@ def main():
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
     rk = dist_setup(args.gpus)
-    if args.workload == "c5":
-        out, host = bench_linear(args, rk)
-    elif args.workload == "soft":
-        out, host = bench_soft(args, rk)
-    elif args.workload == "kl":
-        out, host = bench_kl(args, rk)
-    else:
-        out, host = bench_rows(args, rk)
+    out, host = run_workload(args, rk, args.workload)
     if rk.rank == 0 and rk.world == 1 and not args.no_cpu_baseline:
         v, unit, cores, sample = oracle_baseline(args.workload, 12.0, host)
         out["cpu_baseline"] = {"value": round(v, 4), "unit": unit, "cores": cores,
                                "kind": "oracle", "sample": sample}
+    host = None
+    also = args.also
+    if also is None:
+        also = ",".join(EXTRA_WORKLOADS) if args.workload == "c2" and not args.rows else "none"
+    extra = [w for w in also.split(",") if w and w != "none" and w != args.workload]
+    if extra:
+        out["workloads"] = {}
+        sub = argparse.Namespace(**vars(args))
+        sub.rows = 0
+        sub.steps = min(args.steps, 20)
+        sub.warmup = max(3, min(args.warmup, 5))
+        for w in extra:
+            sub.workload = w
+            o, _ = run_workload(sub, rk, w)
+            out["workloads"][w] = workload_summary(o)
+            release_device_memory()
     if rk.group is not None:
         rk.group.barrier()
         rk.group.destroy_process_group()

@@ -91,3 +91,21 @@ def test_clock_summary_reports_slowdowns_and_missing_samples(tmp_path):
     assert sampler(tmp_path, ["nothing useful\n"]).summary() is None
     cs = bench.ClockSampler(0)  # nvidia-smi never started
     assert cs.summary() is None
+
+
+def test_roofline_reports_measured_and_spec_fractions():
+    r = bench.roofline("hbm", "backward", 6000.0, 6547.2, "measured", None, 123)
+    assert r["frac"] == round(6000.0 / 6547.2, 4) and r["unit"] == "GB/s"
+    assert r["spec_peak"] == 8000.0 and r["frac_of_spec"] == 0.75
+    assert r["algorithmic_bytes_per_launch"] == 123
+    t = bench.roofline("tensor", "forward", 1125.0, 1383.8, "measured (sustained)", 5, 7)
+    assert t["unit"] == "TFLOP/s" and t["frac_of_spec"] == 0.5 and t["traffic"] == 5
+    assert t["algorithmic_flop_per_launch"] == 7
+
+
+def test_workload_summary_keeps_the_rates_and_evidence():
+    line = {"metric": "m", "value": 1.0, "unit": "GB/s", "n_gpus": 1, "fwd_GBs": 2.0,
+            "roofline": {"frac": 0.5}, "clocks": {"sm_mhz": 1965.0}, "e2e": {"value": 0.1},
+            "config": {"workload": "c3a"}, "cpu_baseline": {"value": 1}}
+    s = bench.workload_summary(line)
+    assert set(s) == {"value", "unit", "fwd_GBs", "roofline", "clocks", "e2e", "config"}
