@@ -705,6 +705,9 @@ def bench_linear(args, rk):
     dom, dom_ms, dom_flop = ("backward", bwd_ms, bwd_flop) if bwd_ms >= fwd_ms else \
         ("forward", fwd_ms, fwd_flop)
     achieved = dom_flop / (dom_ms * 1e-3) / 1e12
+    ws_sizes = {"forward": int(ws_f.numel()), "backward": int(ws_b.numel())}
+    del ws_f, ws_b
+    dvf = dense_vs_fused(H, W, yd, g, steps=3)
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
@@ -712,7 +715,7 @@ def bench_linear(args, rk):
         "data": "synthetic",
         "fwd_tflops": round(fwd_flop / (fwd_ms * 1e-3) / 1e12, 2), "fwd_ms": round(fwd_ms, 4),
         "bwd_ms": round(bwd_ms, 4),
-        "workspace_bytes": {"forward": int(ws_f.numel()), "backward": int(ws_b.numel())},
+        "workspace_bytes": ws_sizes,
         "config": {"workload": f"c5: fused linear CE, H ({N}, {D}) bf16 ~N(0,1), W ({V}, {D}) "
                                "bf16 ~N(0, std 0.02), forward + backward (logits recomputed)",
                    "N": N, "V": V, "D": D, "flop_per_step": step_flop,
@@ -724,10 +727,69 @@ def bench_linear(args, rk):
         "roofline": roofline("tensor", dom, achieved, peak_sust, src + " (sustained)",
                              recorded_traffic("c5", dom), dom_flop),
     }
+    out["dense_vs_fused"] = dvf
     clocks = clk.summary()
     if clocks:
         out["clocks"] = clocks
     return out, None
+
+
+def dense_vs_fused(H, W, y, g, steps: int = 3) -> dict:
+    """The comparison of Ineshin's section 3 on the same inputs: time and peak
+    device memory of one forward + backward step, (a) fused (Z = H W^T never
+    stored; this library) and (b) materialised: Z computed by a library GEMM
+    (torch.matmul, cuBLAS) and stored in bf16, the row kernels of this library
+    on it (the gradient written over Z), and library GEMMs for dH = G W and
+    dW = G^T H. Arm (b) is a comparison arm only. Peak memory is what the step
+    allocates on top of H, W, the targets and g: outputs, workspaces, Z."""
+    import torch
+    import softmax_cross_entropy_lse_b200 as ce
+    stream = torch.cuda.current_stream()
+
+    def fused():
+        loss, lse = ce.linear_ce_forward(H, W, y)
+        ev[1].record(stream)
+        dH, dW = ce.linear_ce_backward(g, H, W, y, lse)
+        return loss, dH, dW
+
+    def dense():
+        Z = torch.matmul(H, W.t())
+        r = ce.ce_forward(Z, y)
+        ev[1].record(stream)
+        ce.ce_backward(g, Z, y, r.lse, r.lse_lo, dlogits=Z)
+        dH = torch.matmul(Z, W)
+        dW = torch.matmul(Z.t(), H)
+        return r.loss, dH, dW
+
+    res = {}
+    for name, fn in (("fused", fused), ("materialised", dense)):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        release_device_memory()
+        fn()  # warm-up (library handles, kernel attributes)
+        release_device_memory()
+        base = torch.cuda.memory_allocated()
+        torch.cuda.reset_peak_memory_stats()
+        fwd, bwd = [], []
+        for _ in range(steps):
+            ev[0].record(stream)
+            outs = fn()
+            ev[2].record(stream)
+            torch.cuda.synchronize()
+            fwd.append(ev[0].elapsed_time(ev[1]))
+            bwd.append(ev[1].elapsed_time(ev[2]))
+            del outs
+        peak = torch.cuda.max_memory_allocated() - base
+        res[name] = {"fwd_ms": round(float(np.median(fwd)), 3),
+                     "bwd_ms": round(float(np.median(bwd)), 3),
+                     "step_ms": round(float(np.median(np.add(fwd, bwd))), 3),
+                     "peak_step_bytes": int(peak)}
+    res["fused_speedup"] = round(res["materialised"]["step_ms"] / res["fused"]["step_ms"], 3)
+    res["memory_ratio"] = round(res["materialised"]["peak_step_bytes"] /
+                                max(res["fused"]["peak_step_bytes"], 1), 3)
+    res["note"] = ("materialised arm: Z = H W^T by torch.matmul (cuBLAS) stored in bf16, this "
+                   "library's row forward and VJP on it, dH and dW by torch.matmul; "
+                   "dH and dW in bf16 in both arms")
+    return res
 
 
 # -- CPU oracle ---------------------------------------------------------------------------------
