@@ -339,6 +339,10 @@ def bench_rows(args, rk):
         fwd_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
         bwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
 
+    # the forward alone, back to back: inside the step the forward also pays for
+    # writing back the gradient lines the previous backward left dirty in L2
+    fwd_alone_ms = timed("fwd", args.steps)[0] / args.steps if not use_graph else fwd_ms
+
     # the same step through the fused call (one read of each row that fits on chip)
     fused_ms = timed("fused", args.steps)[0] / args.steps
 
@@ -384,6 +388,7 @@ def bench_rows(args, rk):
         "rows_per_s": round(world * N * args.steps / (ms * 1e-3), 1),
         "fwd_GBs": round(fwd_bytes / (fwd_ms * 1e-3) / 1e9, 2),
         "fwd_rows_per_s": round(N / (fwd_ms * 1e-3), 1),
+        "fwd_alone_GBs": round(fwd_bytes / (fwd_alone_ms * 1e-3) / 1e9, 2),
         "bwd_GBs": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9, 2),
         "config": {"workload": f"{args.workload}: {spec['desc']}; forward + backward",
                    "rows": N, "classes": V, "label_smoothing": eps, "ignore_index": -100,
@@ -982,7 +987,7 @@ def run_reference(args):
 
 EXTRA_WORKLOADS = ["c1", "c3a", "c3b", "c4a", "c4b", "c5", "soft", "kl"]
 SUMMARY_KEYS = ("value", "unit", "ms_per_step", "steps", "dtype", "rows_per_s", "fwd_GBs",
-                "fwd_rows_per_s", "bwd_GBs", "fwd_tflops", "fwd_ms", "bwd_ms", "workspace_bytes",
+                "fwd_rows_per_s", "fwd_alone_GBs", "bwd_GBs", "fwd_tflops", "fwd_ms", "bwd_ms", "workspace_bytes",
                 "vs_baseline", "vs_baseline_basis", "gpu_launches", "roofline", "fused", "clocks",
                 "e2e", "config", "dense_vs_fused")
 

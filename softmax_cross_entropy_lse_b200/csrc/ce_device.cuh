@@ -438,6 +438,62 @@ __device__ __forceinline__ void fold_raw16(OnlineState& st, const uint4 (&w)[U],
     }
 }
 
+// ---- folding against a fixed reference ------------------------------------------
+// Once a lane's state has a finite running max m (its first part folded the
+// exact way), later parts need neither their max nor a rescale: any
+// reference point gives the same log-sum-exp, lse = m + log sum_j exp(z_j - m),
+// as long as no term overflows. Each element then costs one fused
+// multiply-add for its exponent,
+//     a_j = z_j log2 e - mL,   mL = m log2 e rounded to float,
+// and one base-2 exponential. The product m log2 e is not exact: with the
+// exact residual r = m log2 e - mL (an fma recovers it), z_j log2 e - mL =
+// (z_j - m) log2 e + r, so the part's sum carries the common factor 2^r,
+// removed once per part by c = 2^-r. The reference is used only while
+// |m| <= 2^23, where |r| <= 1/2 and the single rounding of a_j costs no more
+// than the two roundings of (z_j - m) log2 e. A part whose sum exceeds 2^100
+// (a term far above the reference) or is not a number is refused, and the
+// caller folds it the exact way, which rescales the state to the part's max.
+struct FoldRef {
+    float mL;  // m log2 e rounded to float
+    float c;   // 2^-(m log2 e - mL)
+    bool ok;   // the reference may be used
+};
+
+__device__ __forceinline__ FoldRef fold_ref(const OnlineState& st) {
+    FoldRef f;
+    f.ok = fabsf(st.m) <= 8388608.f;  // false for an infinite or NaN max
+    f.mL = f.ok ? st.m * kLog2e : 0.f;
+    f.c = f.ok ? ex2(-fmaf(st.m, kLog2e, -f.mL)) : 1.f;
+    return f;
+}
+
+// Folds U 16-byte words of 8 16-bit values (all valid) into (m, s) against the
+// reference f. Returns false, leaving the state unchanged, when the part must
+// be folded the exact way instead. t and k are not kept (no label smoothing).
+template <typename T, int U>
+__device__ __forceinline__ bool fold_raw16_ref(OnlineState& st, const uint4 (&w)[U],
+                                               const FoldRef& f) {
+    using R = Raw16<T>;
+    const float2 l2 = make_float2(kLog2e, kLog2e);
+    const float2 nmL = make_float2(-f.mL, -f.mL);
+    float2 sa = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const uint32_t ws[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+        float2 su = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 a = __ffma2_rn(R::widen(ws[k]), l2, nmL);
+            su = __fadd2_rn(su, make_float2(ex2(a.x), ex2(a.y)));
+        }
+        sa = __fadd2_rn(sa, su);
+    }
+    const float sp = sa.x + sa.y;
+    if (!(sp <= 1.2676506e30f)) return false;  // 2^100; NaN fails too
+    st.s = fmaf(sp, f.c, st.s);
+    return true;
+}
+
 // A whole row of NV 16-byte words (n = NV * VEC values, all valid) folded in
 // one piece: its max first, then the sum of exponentials, with no running
 // state to rescale. The sums go per vector, then across vectors: the order

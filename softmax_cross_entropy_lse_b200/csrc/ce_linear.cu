@@ -17,10 +17,13 @@
 //    consecutive vocabulary tiles, kept in registers, then a partial state
 //    per (unit, row) merged in unit order by a second launch;
 //  * backward: for each vocabulary chunk, GEMM 1 recomputes Z_c = H W_c^T and
-//    its epilogue writes G_c = g (softmax - (1-eps) onehot - eps/V) in bf16
-//    (row-major and transposed); GEMM 2 forms dW_c = G_c^T H; GEMM 3 adds
-//    G_c W_c into a float dH accumulator. Each dW row belongs to one chunk,
-//    so dW needs no accumulation across chunks.
+//    its epilogue writes G_c = g (softmax - (1-eps) onehot - eps/V) in bf16;
+//    GEMM 2 forms dW_c = G_c^T H; GEMM 3 adds G_c W_c into a float dH
+//    accumulator. Each dW row belongs to one chunk, so dW needs no
+//    accumulation across chunks. GEMM 2 reads both its operands, and GEMM 3
+//    its B operand, in their stored orientation: the tiles are loaded
+//    MN-major (the output index contiguous) and the MMA descriptors say so,
+//    so no transposed copy of H, W or G_c is ever made.
 // Every pipeline wait is bounded in time; on expiry the CTA raises an error
 // bit, drains its own copies and MMAs, frees its tensor memory and returns.
 #include <cudaTypedefs.h>
@@ -42,7 +45,17 @@ constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr int kGemmThreads = 192;  // warp 0: TMA, warp 1: MMA, warps 2-5: epilogue
 constexpr uint32_t kTmemCols = 2 * kBN;
 constexpr size_t kGemmSmem = 1024 + (size_t)kStages * kStageBytes + 256;
-constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN);
+// An MN-major operand tile arrives as boxes of 64 (M or N) x kBK (K) elements,
+// 8 KB each, stacked along M/N.
+constexpr int kMnBox = 64;
+constexpr uint32_t kMnBoxBytes = kMnBox * kBK * 2;
+// Reach of one MMA's MN-major descriptor: its start moves 2 KB per K step of
+// 16, it spans the tile's boxes along M/N (leading offset) and two 1 KB K
+// groups (stride offset). The last byte must stay inside the stage's tile.
+static_assert((kBK / 16 - 1) * 2048 + (kBM / kMnBox - 1) * kMnBoxBytes + 2048 <= kABytes,
+              "an MN-major A descriptor reaches past its stage");
+static_assert((kBK / 16 - 1) * 2048 + (kBN / kMnBox - 1) * kMnBoxBytes + 2048 <= kBBytes,
+              "an MN-major B descriptor reaches past its stage");
 
 enum EpiKind { kEpiCeFwd = 0, kEpiCeGrad = 1, kEpiStore = 2, kEpiAccum = 3 };
 
@@ -69,8 +82,6 @@ struct GemmArgs {
     const float* lse;
     __nv_bfloat16* G;          // gradient chunk, row-major, ld = ldG
     int64_t ldG;
-    __nv_bfloat16* GT;         // its transpose, ld = ldGT
-    int64_t ldGT;
     // store / accumulate epilogues
     void* C;                   // output rows start here
     int64_t ldc;
@@ -140,12 +151,16 @@ __device__ __forceinline__ void store_row32(void* base, int64_t ld, int64_t row,
 }
 
 // ---------------------------------------------------------------------------
-// The persistent GEMM: C[M x Nn] = A[M x K] * B[Nn x K]^T, bf16 K-major
-// operands through TMA tensor maps, f32 accumulation in tensor memory.
-template <int EPI>
+// The persistent GEMM: C[M x Nn] = A[M x K] * B[Nn x K]^T, bf16 operands
+// through TMA tensor maps, f32 accumulation in tensor memory. An operand is
+// K-major (its K index contiguous in memory: A as M x K, B as Nn x K, loaded
+// in 64-wide boxes of K) or, with AMN / BMN, MN-major (its M or Nn index
+// contiguous: A stored K x M, B stored K x Nn, loaded in 64 x 64 boxes).
+template <int EPI, bool AMN, bool BMN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const GemmArgs a) {
+    constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN, AMN, BMN);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -211,10 +226,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         // the MMA thread's wait for this stage runs out)
                         if (!a.starve) {
                             mbar_expect_tx(full_bar(s), kStageBytes);
-                            tma_load_2d(smem_u32(sA + s * kABytes), &tmA, full_bar(s),
-                                        a.kA0 + kb * kBK, mb * kBM);
-                            tma_load_2d(smem_u32(sB + s * kBBytes), &tmB, full_bar(s),
-                                        a.kB0 + kb * kBK, nb * kBN);
+                            const int k0a = a.kA0 + kb * kBK, k0b = a.kB0 + kb * kBK;
+                            if constexpr (AMN) {
+#pragma unroll
+                                for (int h = 0; h < kBM / kMnBox; ++h)
+                                    tma_load_2d(smem_u32(sA + s * kABytes + h * kMnBoxBytes), &tmA,
+                                                full_bar(s), mb * kBM + h * kMnBox, k0a);
+                            } else {
+                                tma_load_2d(smem_u32(sA + s * kABytes), &tmA, full_bar(s), k0a,
+                                            mb * kBM);
+                            }
+                            if constexpr (BMN) {
+#pragma unroll
+                                for (int h = 0; h < kBN / kMnBox; ++h)
+                                    tma_load_2d(smem_u32(sB + s * kBBytes + h * kMnBoxBytes), &tmB,
+                                                full_bar(s), nb * kBN + h * kMnBox, k0b);
+                            } else {
+                                tma_load_2d(smem_u32(sB + s * kBBytes), &tmB, full_bar(s), k0b,
+                                            nb * kBN);
+                            }
                             issued_mask |= 1u << s;
                             last_ph = (last_ph & ~(1u << s)) | (ph << s);
                         }
@@ -259,11 +289,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         tc_fence_after();
                         const uint32_t a0 = smem_u32(sA + s * kABytes);
                         const uint32_t b0 = smem_u32(sB + s * kBBytes);
+                        // K steps of 16: 32 bytes along a K-major row, two
+                        // 8-row K groups (2 KB) down an MN-major atom column
 #pragma unroll
-                        for (int kk = 0; kk < kBK / 16; ++kk)
-                            umma_bf16(d, desc_kmajor_sw128(a0 + kk * 32),
-                                      desc_kmajor_sw128(b0 + kk * 32), kIdesc,
-                                      (kb | kk) != 0 ? 1u : 0u);
+                        for (int kk = 0; kk < kBK / 16; ++kk) {
+                            const uint64_t da = AMN ? desc_mnmajor_sw128(a0 + kk * 2048, kMnBoxBytes)
+                                                    : desc_kmajor_sw128(a0 + kk * 32);
+                            const uint64_t db = BMN ? desc_mnmajor_sw128(b0 + kk * 2048, kMnBoxBytes)
+                                                    : desc_kmajor_sw128(b0 + kk * 32);
+                            umma_bf16(d, da, db, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                        }
                         umma_commit(empty_bar(s));
                         if (++s == kStages) {
                             s = 0;
@@ -359,13 +394,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             v[j] = gv;
                         }
                         if (row_ok) store_row32(a.G, a.ldG, m, c, v, 0, nv);
-                        // transposed copy: column j of this chunk is row c + j of
-                        // G^T; the 32 lanes write 32 consecutive rows' entries
-                        if (row_ok) {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if (j < nv) a.GT[(c + j) * a.ldGT + m] = __float2bfloat16_rn(v[j]);
-                        }
                     } else if constexpr (EPI == kEpiStore) {
                         if (row_ok) store_row32(a.C, a.ldc, m, c, v, a.c_f32, nv);
                     } else {  // kEpiAccum
@@ -443,29 +471,6 @@ __global__ void __launch_bounds__(256) k_linear_merge(const float4* part, int64_
     }
 }
 
-// dst[c][r] = src[r][c] for a rows x cols bf16 matrix (both 2-byte elements).
-__global__ void __launch_bounds__(256) k_transpose_bf16(const __nv_bfloat16* src, int64_t ld_src,
-                                                        __nv_bfloat16* dst, int64_t ld_dst,
-                                                        int64_t rows, int64_t cols) {
-    __shared__ __nv_bfloat16 tile[64][65];
-    const int64_t tiles_c = (cols + 63) / 64;
-    const int64_t ntiles = ((rows + 63) / 64) * tiles_c;
-    const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 64 x 4
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
-        const int64_t r0 = (t / tiles_c) * 64, c0 = (t % tiles_c) * 64;
-        for (int i = ty; i < 64; i += 4) {
-            const int64_t r = r0 + i, c = c0 + tx;
-            tile[i][tx] = (r < rows && c < cols) ? src[r * ld_src + c] : __float2bfloat16_rn(0.f);
-        }
-        __syncthreads();
-        for (int i = ty; i < 64; i += 4) {
-            const int64_t c = c0 + i, r = r0 + tx;
-            if (c < cols && r < rows) dst[c * ld_dst + r] = tile[tx][i];
-        }
-        __syncthreads();
-    }
-}
-
 // ---------------------------------------------------------------------------
 // Host side.
 
@@ -484,7 +489,9 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // Tensor map of a row-major bf16 matrix (rows x cols, row stride ld elements)
-// loaded in boxes of 64 columns x box_rows rows with 128-byte swizzle.
+// loaded in boxes of 64 columns x box_rows rows with 128-byte swizzle (the
+// row of a box is 128 bytes, one swizzle row). Out-of-range elements read as
+// zero.
 static bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ld,
                      int box_rows) {
     auto enc = encode_fn();
@@ -499,10 +506,10 @@ static bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t c
     return r == CUDA_SUCCESS;
 }
 
-template <int EPI>
+template <int EPI, bool AMN = false, bool BMN = false>
 static cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmArgs a, int sms,
                                cudaStream_t s) {
-    cudaError_t e = ensure_smem_limit((const void*)k_gemm<EPI>, (int)kGemmSmem);
+    cudaError_t e = ensure_smem_limit((const void*)k_gemm<EPI, AMN, BMN>, (int)kGemmSmem);
     if (e != cudaSuccess) return e;
     const WaitPolicy wp = wait_policy();
     a.wait_ns = wp.limit_ns;
@@ -514,14 +521,19 @@ static cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, Gem
     a.n_units_n = (a.n_nb + a.tiles_per_unit - 1) / a.tiles_per_unit;
     a.units = (int64_t)a.n_mb * a.n_units_n;
     const int grid = (int)(a.units < sms ? a.units : sms);
-    k_gemm<EPI><<<grid, kGemmThreads, kGemmSmem, s>>>(ta, tb, a);
+    k_gemm<EPI, AMN, BMN><<<grid, kGemmThreads, kGemmSmem, s>>>(ta, tb, a);
     return cudaGetLastError();
 }
 
 // Vocabulary tiles per forward unit: a few, so the W tiles in use by all CTAs
 // at once stay in L2 next to H.
 static constexpr int kFwdTilesPerUnit = 4;
-static constexpr int64_t kBwdChunk = 8192;  // vocabulary columns per backward chunk
+// Vocabulary columns per backward chunk (a multiple of the 256-column tile).
+#ifndef CE_BWD_CHUNK
+#define CE_BWD_CHUNK 8192
+#endif
+static constexpr int64_t kBwdChunk = CE_BWD_CHUNK;
+static_assert(kBwdChunk % kBN == 0, "whole output tiles per chunk");
 
 static int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
@@ -536,27 +548,24 @@ static size_t fwd_ws(int64_t N, int64_t V) {
     return (size_t)units * (size_t)N * sizeof(float4);
 }
 
+// Backward workspace: one vocabulary chunk of the logits' gradient (bf16,
+// row-major N x vc) and the float dH accumulator (N x D; not needed when dH
+// itself is float).
 struct BwdLayout {
-    size_t off_ht, off_wt, off_g, off_gt, off_acc, total;
-    int64_t ld_ht, ld_wt, vc, ld_gt;
+    size_t off_g, off_acc, total;
+    int64_t vc;
 };
 
 static BwdLayout bwd_layout(int64_t N, int64_t V, int64_t D) {
     BwdLayout L{};
-    L.ld_ht = round_up(N, 8);
     L.vc = V < kBwdChunk ? round_up(V, kBN) : kBwdChunk;
-    L.ld_wt = L.vc;  // one vocabulary chunk of W^T at a time
-    L.ld_gt = round_up(N, 8);
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t o = off;
         off = (size_t)round_up((int64_t)(off + bytes), 256);
         return o;
     };
-    L.off_ht = take((size_t)D * L.ld_ht * 2);
-    L.off_wt = take((size_t)D * L.vc * 2);
     L.off_g = take((size_t)N * L.vc * 2);
-    L.off_gt = take((size_t)L.vc * L.ld_gt * 2);
     L.off_acc = take((size_t)N * D * 4);
     L.total = off;
     return L;
@@ -646,42 +655,25 @@ ce_status linear_ce_backward(const float* grad_out, int64_t grad_stride, const v
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
     const int sms = device_sms(0);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    auto* HT = reinterpret_cast<__nv_bfloat16*>(ws + L.off_ht);
-    auto* WT = reinterpret_cast<__nv_bfloat16*>(ws + L.off_wt);
     auto* G = reinterpret_cast<__nv_bfloat16*>(ws + L.off_g);
-    auto* GT = reinterpret_cast<__nv_bfloat16*>(ws + L.off_gt);
     float* dH_acc = dH_dt == CE_F32 ? static_cast<float*>(dH) : reinterpret_cast<float*>(ws + L.off_acc);
 
-    // transposed copy of H (the K-major B operand of the dW pass); W is
-    // transposed one vocabulary chunk at a time below
-    {
-        const int64_t t1 = ((N + 63) / 64) * ((D + 63) / 64);
-        k_transpose_bf16<<<(int)(t1 < (int64_t)sms * 8 ? t1 : (int64_t)sms * 8), 256, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(H), ld_h, HT, L.ld_ht, N, D);
-        if (cudaGetLastError() != cudaSuccess) return CE_ECUDA;
-    }
-    CUtensorMap mH, mHT;
-    if (!make_map(&mH, H, N, D, ld_h, kBM) || !make_map(&mHT, HT, D, N, L.ld_ht, kBN))
+    // H as the K-major A operand of GEMM 1 and as the MN-major B operand of
+    // GEMM 2 (its rows are the reduction index there)
+    CUtensorMap mH, mHmn;
+    if (!make_map(&mH, H, N, D, ld_h, kBM) || !make_map(&mHmn, H, N, D, ld_h, kMnBox))
         return CE_ECUDA;
 
     const int64_t nchunks = (V + L.vc - 1) / L.vc;
     for (int64_t c = 0; c < nchunks; ++c) {
         const int64_t v0 = c * L.vc;
         const int64_t vcv = (V - v0) < L.vc ? (V - v0) : L.vc;  // valid columns
-        // W_c^T (D x vcv, leading dimension vc): the K-major B operand of the
-        // dH pass. Stream order keeps the previous chunk's dH pass ahead of
-        // this overwrite.
-        {
-            const int64_t t2 = ((vcv + 63) / 64) * ((D + 63) / 64);
-            k_transpose_bf16<<<(int)(t2 < (int64_t)sms * 8 ? t2 : (int64_t)sms * 8), 256, 0, s>>>(
-                static_cast<const __nv_bfloat16*>(W) + v0 * ld_w, ld_w, WT, L.ld_wt, vcv, D);
-            if (cudaGetLastError() != cudaSuccess) return CE_ECUDA;
-        }
-        // GEMM 1: Z_c = H W_c^T, epilogue writes G_c and G_c^T
+        const __nv_bfloat16* Wc = static_cast<const __nv_bfloat16*>(W) + v0 * ld_w;
+        // GEMM 1: Z_c = H W_c^T, epilogue writes G_c (stream order keeps the
+        // previous chunk's GEMMs, which read G_c, ahead of this overwrite)
         {
             CUtensorMap mWc;
-            if (!make_map(&mWc, static_cast<const __nv_bfloat16*>(W) + v0 * ld_w, vcv, D, ld_w, kBN))
-                return CE_ECUDA;
+            if (!make_map(&mWc, Wc, vcv, D, ld_w, kBN)) return CE_ECUDA;
             GemmArgs a{};
             a.M = (int)N;
             a.Nn = (int)vcv;
@@ -699,14 +691,15 @@ ce_status linear_ce_backward(const float* grad_out, int64_t grad_stride, const v
             a.lse = lse;
             a.G = G;
             a.ldG = L.vc;
-            a.GT = GT;
-            a.ldGT = L.ld_gt;
             if (launch_gemm<kEpiCeGrad>(mH, mWc, a, sms, s) != cudaSuccess) return CE_ECUDA;
         }
-        // GEMM 2: dW[v0:v0+vcv] = G_c^T H  (A = G_c^T, B = H^T, K = N)
+        // GEMM 2: dW[v0:v0+vcv] = G_c^T H (M = vcv, K = N): A is G_c read with
+        // its vocabulary index contiguous, B is H read with D contiguous, both
+        // MN-major. The maps stop at vcv columns, so the stale columns of the
+        // last, narrower chunk read as zero.
         {
-            CUtensorMap mGT;
-            if (!make_map(&mGT, GT, vcv, N, L.ld_gt, kBM)) return CE_ECUDA;
+            CUtensorMap mGmn;
+            if (!make_map(&mGmn, G, N, vcv, L.vc, kMnBox)) return CE_ECUDA;
             GemmArgs a{};
             a.M = (int)vcv;
             a.Nn = (int)D;
@@ -717,12 +710,14 @@ ce_status linear_ce_backward(const float* grad_out, int64_t grad_stride, const v
             a.C = static_cast<uint8_t*>(dW) + (size_t)v0 * D * esz;
             a.ldc = D;
             a.c_f32 = dW_dt == CE_F32;
-            if (launch_gemm<kEpiStore>(mGT, mHT, a, sms, s) != cudaSuccess) return CE_ECUDA;
+            if (launch_gemm<kEpiStore, true, true>(mGmn, mHmn, a, sms, s) != cudaSuccess)
+                return CE_ECUDA;
         }
-        // GEMM 3: dH (+)= G_c W_c  (A = G_c, B = W_c^T, K = vcv)
+        // GEMM 3: dH (+)= G_c W_c (K = vcv): A is G_c K-major, B is W_c read
+        // with D contiguous (MN-major)
         {
-            CUtensorMap mG, mWT;
-            if (!make_map(&mG, G, N, vcv, L.vc, kBM) || !make_map(&mWT, WT, D, vcv, L.ld_wt, kBN))
+            CUtensorMap mG, mWmn;
+            if (!make_map(&mG, G, N, vcv, L.vc, kBM) || !make_map(&mWmn, Wc, vcv, D, ld_w, kMnBox))
                 return CE_ECUDA;
             GemmArgs a{};
             a.M = (int)N;
@@ -739,7 +734,8 @@ ce_status linear_ce_backward(const float* grad_out, int64_t grad_stride, const v
             a.C = dH;
             a.ldc = D;
             a.c_f32 = dH_dt == CE_F32;
-            if (launch_gemm<kEpiAccum>(mG, mWT, a, sms, s) != cudaSuccess) return CE_ECUDA;
+            if (launch_gemm<kEpiAccum, false, true>(mG, mWmn, a, sms, s) != cudaSuccess)
+                return CE_ECUDA;
         }
     }
     return CE_OK;

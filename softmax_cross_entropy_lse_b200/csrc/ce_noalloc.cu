@@ -27,7 +27,7 @@ namespace {
 constexpr size_t kScratchBytes = CE_NOALLOC_SCRATCH_BYTES;  // 64 KiB per device
 constexpr int kMaxDevices = 64;
 
-__device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 std::mutex g_scratch_mutex;
 void* g_scratch_ptr[kMaxDevices];

@@ -54,9 +54,11 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, const uint4& v
         : "memory");
 }
 
+// Folds one chunk. 16-bit rows without argmax or label smoothing fold every
+// chunk after a lane's first against the lane's reference max (ref).
 template <typename TI, bool ARGMAX, bool WITH_T>
-__device__ __forceinline__ void fold_chunk(OnlineState& st, const uint4* buf, int nvc, int lane,
-                                           int64_t col_vec0) {
+__device__ __forceinline__ void fold_chunk(OnlineState& st, FoldRef& ref, const uint4* buf, int nvc,
+                                           int lane, int64_t col_vec0) {
     constexpr int VEC = ElemTraits<TI>::kVec;
     constexpr int kPerLane = kSmChunkVecs / 32;
     if constexpr (sizeof(TI) == 2 && !ARGMAX) {
@@ -68,10 +70,19 @@ __device__ __forceinline__ void fold_chunk(OnlineState& st, const uint4* buf, in
             ok[q] = vi < nvc;
             if (ok[q]) w[q] = buf[vi];
         }
-        if (nvc == kSmChunkVecs)
-            fold_raw16<TI, kPerLane, false, WITH_T>(st, w, ok);
-        else
+        if (nvc == kSmChunkVecs) {
+            bool done = false;
+            if constexpr (!WITH_T) {
+                if (ref.ok) done = fold_raw16_ref<TI, kPerLane>(st, w, ref);
+            }
+            if (!done) {
+                fold_raw16<TI, kPerLane, false, WITH_T>(st, w, ok);
+                if constexpr (!WITH_T) ref = fold_ref(st);
+            }
+        } else {
             fold_raw16<TI, kPerLane, true, WITH_T>(st, w, ok);
+            if constexpr (!WITH_T) ref = fold_ref(st);
+        }
     } else {
         float v[kPerLane][VEC];
         bool ok[kPerLane];
@@ -217,6 +228,8 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
 
         // ---- forward: fold the slice as its chunks land
         OnlineState st = empty_state();
+        FoldRef ref;
+        ref.ok = false;
         for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps) {
             if (!dead) {
                 if (mbar_wait(smem_u32(&full_bar[c]), (phase >> i) & 1u, &abort_flag)) {
@@ -227,7 +240,7 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
                 }
             }
             if (!dead)
-                fold_chunk<TI, ARGMAX, WITH_T>(st, chunk_buf(c), chunk_vecs(c), lane,
+                fold_chunk<TI, ARGMAX, WITH_T>(st, ref, chunk_buf(c), chunk_vecs(c), lane,
                                                v0 + (int64_t)c * kSmChunkVecs);
         }
         if (tail_here) {

@@ -452,6 +452,8 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
             if (y != a.ignore && y >= 0 && y < a.V) zy = to_f32(row[y]);
         }
         OnlineState st = empty_state();
+        FoldRef ref;
+        ref.ok = false;  // the unit's first part is folded the exact way
         for (int j = wid; j < ru.nch; j += kRingWarps) {
             const int stage = (int)(consumed & (kRingStages - 1));
             const uint32_t bar = smem_u32(&full_bar[wid][stage]);
@@ -480,10 +482,21 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
                             ok[q] = vi < nvh;
                             if (ok[q]) w[q] = buf[vi];
                         }
-                        if (nvh == kRingPart)
-                            fold_raw16<T, kPerLane, false, WITH_T>(st, w, ok);
-                        else
+                        if (nvh == kRingPart) {
+                            // without label smoothing, parts after the first
+                            // fold against the lane's reference max
+                            bool done = false;
+                            if constexpr (!WITH_T) {
+                                if (ref.ok) done = fold_raw16_ref<T, kPerLane>(st, w, ref);
+                            }
+                            if (!done) {
+                                fold_raw16<T, kPerLane, false, WITH_T>(st, w, ok);
+                                if constexpr (!WITH_T) ref = fold_ref(st);
+                            }
+                        } else {
                             fold_raw16<T, kPerLane, true, WITH_T>(st, w, ok);
+                            if constexpr (!WITH_T) ref = fold_ref(st);
+                        }
                     } else {
                         float v[kPerLane][VEC];
                         bool ok[kPerLane];

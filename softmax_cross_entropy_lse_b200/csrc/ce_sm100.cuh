@@ -12,9 +12,14 @@
 //     1024-byte swizzle atoms: the stride between 8-row groups is 1024 bytes,
 //     the leading offset is unused (1). Stepping K by 16 elements inside the
 //     atom adds 32 bytes to the start address.
+//     An MN-major tile (the M or N index contiguous, as in a row-major
+//     operand read along its columns) is a grid of 1024-byte atoms of 8 rows
+//     of K x 128 bytes (64 bf16 of M or N): the leading byte offset is the
+//     stride between atoms along M/N, the stride byte offset the stride
+//     between groups of 8 K. Stepping K by 16 elements moves two K groups.
 //   instruction descriptor: D format in [4,6) (1 = f32), A and B formats in
-//     [7,10) and [10,13) (1 = bf16), A/B major in bits 15/16 (0 = K-major),
-//     N >> 3 in [17,23), M >> 4 in [24,29).
+//     [7,10) and [10,13) (1 = bf16), A/B major in bits 15/16 (0 = K-major,
+//     1 = MN-major), N >> 3 in [17,23), M >> 4 in [24,29).
 #pragma once
 
 #include <cuda.h>
@@ -260,10 +265,25 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t smem_addr) {
     return d;
 }
 
-// kind::f16 instruction descriptor: bf16 x bf16 -> f32, both K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
+// MN-major, 128-byte swizzle: atoms of 8 K-rows x 128 bytes; `lbo` bytes
+// between atoms along M/N, 1024 bytes between groups of 8 K (the atoms of one
+// 64-wide M/N slice are stacked along K).
+__device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t smem_addr, uint32_t lbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;  // leading byte offset: next 64 of M/N
+    d |= (uint64_t)(1024 >> 4) << 32;             // stride byte offset: next 8 of K
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// kind::f16 instruction descriptor: bf16 x bf16 -> f32; A and B K-major unless
+// a_mn / b_mn mark them MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn = false,
+                                                      bool b_mn = false) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
+           ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 }  // namespace sm100
