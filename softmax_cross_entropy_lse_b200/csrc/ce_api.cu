@@ -190,11 +190,15 @@ static FwdPlan plan_forward(int64_t N, int64_t V, int esz, bool vec_ok, int sms)
         const int64_t cap = (int64_t)sms * 16;
         p.grid = (int)(want < cap ? (want > 0 ? want : 1) : cap);
         // whole-vector 4-byte rows that one step covers: pipelined through
-        // shared memory, three resident blocks per SM, every block resident
-        if (vec_ok && esz == 4 && p.G >= 2 && V % p.vec == 0 && nvec <= (int64_t)p.G * 8) {
+        // shared memory, three resident blocks per SM, every block resident;
+        // only when every warp gets at least two row groups (with fewer there
+        // is nothing to overlap, and the kernel above takes the batch in one
+        // wave of up to four blocks per SM)
+        const int64_t capp = (int64_t)sms * 3;
+        if (vec_ok && esz == 4 && p.G >= 2 && V % p.vec == 0 && nvec <= (int64_t)p.G * 8 &&
+            want >= 2 * capp) {
             p.pipe = 1;
-            const int64_t capp = (int64_t)sms * 3;
-            p.grid = (int)(want < capp ? (want > 0 ? want : 1) : capp);
+            p.grid = (int)capp;
         }
         return p;
     }
@@ -538,10 +542,29 @@ ce_status ce_soft_backward(const float* grad_out, int64_t grad_stride, const voi
 static KlPlan plan_kl(int64_t N, int64_t V, int esz, bool vec_ok, int sms) {
     KlPlan p = plan_soft(N, V, esz, esz, vec_ok, sms);
     p.cta = 0;
+    p.cl = 1;
+    p.sms = sms;
     if (p.G == 32 && N < (int64_t)sms * 24) {
         p.cta = 1;
         const int64_t cap = (int64_t)sms * 4;
         p.grid = (int)(N < cap ? (N > 0 ? N : 1) : cap);
+        // rows split over a cluster of CL CTAs when that fills the CTA slots
+        // better (4 per SM for 4-byte rows, 3 for 16-bit): the CL with the
+        // fullest last wave, each CTA keeping at least 1024 vectors
+        const int64_t nv = V / p.vec;
+        const int64_t slots = (int64_t)sms * (esz == 4 && p.vec > 1 ? 4 : (p.vec == 1 ? 2 : 3));
+        double best = 0.0;
+        for (int cl = 1; cl <= 8; cl *= 2) {
+            if (cl > 1 && nv / cl < 1024) break;
+            const int64_t ncl = slots / cl;
+            const int64_t waves = (N + ncl - 1) / ncl;
+            const double eff = (double)N / (double)(waves * ncl);
+            if (eff > best + 0.02) {
+                best = eff;
+                p.cl = cl;
+            }
+        }
+        p.vec_per_cta = (nv + p.cl - 1) / p.cl;
         const int64_t nvec = V / p.vec;
         const int64_t nch = nvec > 0 ? (nvec + 1023) / 1024 : 1;
         const int64_t want = (N * nch + 7) / 8;

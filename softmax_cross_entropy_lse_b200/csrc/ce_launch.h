@@ -158,6 +158,9 @@ struct SoftPlan {
     int grid;
     int cta;       // KL: long rows, too few of them for a warp each to fill the GPU
     int grid_bwd;  // KL backward over (row, chunk) units
+    int cl;        // KL forward of long rows: CTAs per row (a cluster), 1, 2, 4 or 8
+    int64_t vec_per_cta;  // vectors of a row each CTA of the cluster folds
+    int sms;
 };
 
 cudaError_t launch_soft_forward(const SoftPlan& p, const SoftArgs& a, int dz_t, int dt_t,

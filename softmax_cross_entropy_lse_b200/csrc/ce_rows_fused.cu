@@ -33,6 +33,7 @@ __global__ void __launch_bounds__(256, MINB) k_fwdbwd_rows(FusedArgs fa) {
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int64_t nvec = a.V / VEC;
     const int tail = (int)(a.V - nvec * VEC);
+    const bool full = nvec == (int64_t)G * U;  // every lane's every vector is in the row
     const RowOut out{a.loss, a.lse, a.lse_lo, a.argmax, a.err};
     const float inv_v = 1.f / (float)a.V;
     const float nan = __int_as_float(0x7fc00000);
@@ -65,8 +66,13 @@ __global__ void __launch_bounds__(256, MINB) k_fwdbwd_rows(FusedArgs fa) {
         OnlineState st = empty_state();
         float zy = 0.f;
         if (act) {
-            fold_vecs<U, VEC, true>(st, v, ok);
-            if constexpr (ARGMAX) argmax_vecs<U, VEC, true>(st, v, ok, c0);
+            if (full) {  // every vector valid: the unpredicated fold (same bits)
+                fold_vecs<U, VEC, false>(st, v, ok);
+                if constexpr (ARGMAX) argmax_vecs<U, VEC, false>(st, v, ok, c0);
+            } else {
+                fold_vecs<U, VEC, true>(st, v, ok);
+                if constexpr (ARGMAX) argmax_vecs<U, VEC, true>(st, v, ok, c0);
+            }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const unsigned dy = (unsigned)(yc - c0[u]);

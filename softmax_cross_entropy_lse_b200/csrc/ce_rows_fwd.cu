@@ -117,6 +117,7 @@ __global__ void __launch_bounds__(kPipeWarps * 32, MINB) k_fwd_packed_pipe(FwdAr
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int64_t step = nwarps * kRowsPerStep;
     const int64_t nvec = a.V / VEC;
+    const bool full = nvec == (int64_t)G * U;  // every lane's every slot holds a vector
     const RowOut out{a.loss, a.lse, a.lse_lo, a.argmax, a.err};
     auto slot = [&](int s, int u) { return pipe_smem + ((s * kPipeWarps + wid) * U + u) * 32 + lane; };
     auto issue = [&](int64_t base, int s) {
@@ -152,15 +153,28 @@ __global__ void __launch_bounds__(kPipeWarps * 32, MINB) k_fwd_packed_pipe(FwdAr
             float v[U][VEC];
             bool ok[U];
             int c0[U];
+            if (full) {
+                // every slot holds a vector: no predicates in the fold (the same
+                // operations in the same order as the masked fold, so the same bits)
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int64_t vi = u * G + gl;
-                ok[u] = vi < nvec;
-                c0[u] = (int)(vi * VEC);
-                if (ok[u]) unpack_words<T>(*slot(s, u), v[u]);
+                for (int u = 0; u < U; ++u) {
+                    ok[u] = true;
+                    c0[u] = (u * G + gl) * VEC;
+                    unpack_words<T>(*slot(s, u), v[u]);
+                }
+                fold_vecs<U, VEC, false>(st, v, ok);
+                if constexpr (ARGMAX) argmax_vecs<U, VEC, false>(st, v, ok, c0);
+            } else {
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int64_t vi = u * G + gl;
+                    ok[u] = vi < nvec;
+                    c0[u] = (int)(vi * VEC);
+                    if (ok[u]) unpack_words<T>(*slot(s, u), v[u]);
+                }
+                fold_vecs<U, VEC, true>(st, v, ok);
+                if constexpr (ARGMAX) argmax_vecs<U, VEC, true>(st, v, ok, c0);
             }
-            fold_vecs<U, VEC, true>(st, v, ok);
-            if constexpr (ARGMAX) argmax_vecs<U, VEC, true>(st, v, ok, c0);
         }
         group_reduce<G, ARGMAX>(st);
         if (active && gl == 0) finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);

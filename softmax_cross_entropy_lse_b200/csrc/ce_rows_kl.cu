@@ -19,6 +19,9 @@
 // no slot to reuse (the race that "One barrier short" is about cannot occur).
 #include "ce_device.cuh"
 #include "ce_launch.h"
+#include "ce_sm100.cuh"
+
+#include <mutex>
 
 namespace ceb {
 
@@ -278,6 +281,114 @@ __global__ void __launch_bounds__(kKlCtaWarps * 32, MINB) k_kl_fwd_cta(KlArgs a)
     }
 }
 
+// Long rows split across a thread-block cluster of CL CTAs: CTA k of the
+// cluster folds vectors [k S, (k+1) S) of the row (S = vec_per_cta) with the
+// 8-warp loop above, reduces its warps in shared memory, and stores its
+// (mq, sq, mp, sp, w) state into slot [parity][k] of the cluster's first CTA,
+// which merges the CL states in rank order and writes the row. A batch of a
+// few hundred rows then fills every CTA slot of the GPU (a CTA per row left
+// the last wave part-empty: 512 rows over 592 slots).
+//
+// One cluster barrier per row orders the exchange, split in halves so that
+// no CTA waits at it: after storing its state of row i a CTA arrives (with
+// release), folds row i + 1, then waits (with acquire) for row i's arrivals
+// before storing its state of row i + 1 into the other slot set. The first
+// CTA reads row i's slots after that wait and before arriving for row i + 1;
+// a slot set is written again only for row i + 2, after the wait for row
+// i + 1, which needs that arrival. No slot is rewritten before it is read
+// (the race "One barrier short" describes cannot occur).
+template <typename T, int VEC, int U, int CL, int MINB>
+__global__ void __launch_bounds__(kKlCtaWarps * 32, MINB) k_kl_fwd_cluster(KlArgs a,
+                                                                           int64_t vec_per_cta) {
+    using namespace sm100;
+    __shared__ KlState wslots[2][kKlCtaWarps];
+    __shared__ __align__(16) float cslots[2][CL][8];  // in the first CTA: (mq, sq, mp, sp, w)
+    const T* __restrict__ zs = reinterpret_cast<const T*>(a.zq);
+    const T* __restrict__ zt = reinterpret_cast<const T*>(a.zp);
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    constexpr int kThreads = kKlCtaWarps * 32;
+    const uint32_t rank = cluster_ctarank();
+    const int64_t cid = cluster_id_x(), ncl = cluster_count_x();
+    const int64_t nvec = a.V / VEC;
+    const int tail = rank == CL - 1 ? (int)(a.V - nvec * VEC) : 0;
+    const int64_t v0 = (int64_t)rank * vec_per_cta;
+    const int64_t v1 = min(nvec, v0 + vec_per_cta);
+    // this CTA's two slots in the first CTA's shared memory
+    const uint32_t dst[2] = {mapa_shared(smem_u32(&cslots[0][rank][0]), 0),
+                             mapa_shared(smem_u32(&cslots[1][rank][0]), 0)};
+
+    // the first CTA merges the CL states of row r (slot set par) and writes it
+    auto finish = [&](int64_t r, int par) {
+        if (rank == 0 && wid == 0) {
+            KlState st{-INFINITY, 0.f, -INFINITY, 0.f, 0.f};
+            if (lane < CL) {
+                const float* c = cslots[par][lane];
+                st = KlState{c[0], c[1], c[2], c[3], c[4]};
+            }
+            kl_group_reduce<CL>(st);  // lanes >= CL hold the empty state
+            if (lane == 0) kl_finalize(a, st, r);
+        }
+    };
+
+    int it = 0;
+    int64_t prev = -1;
+    for (int64_t r = cid; r < a.N; r += ncl, ++it) {
+        const int par = it & 1;
+        const T* qr = zs + row_offset(a.lq, r, a.N);
+        const T* pr = zt + row_offset(a.lp, r, a.N);
+        KlState st{-INFINITY, 0.f, -INFINITY, 0.f, 0.f};
+        for (int64_t vb = v0 + tid; vb < v1; vb += (int64_t)kThreads * U) {
+            Raw<T, VEC> rq[U], rp[U];
+            bool ok[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t vi = vb + (int64_t)u * kThreads;
+                ok[u] = vi < v1;
+                if (ok[u]) {
+                    load_raw<T, VEC>(qr, vi * VEC, a.lq.s_col, rq[u]);
+                    load_raw<T, VEC>(pr, vi * VEC, a.lp.s_col, rp[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (!ok[u]) continue;
+                float q[VEC], p[VEC];
+                unpack_raw<T, VEC>(rq[u], q);
+                unpack_raw<T, VEC>(rp[u], p);
+                kl_fold<VEC>(st, q, p);
+            }
+        }
+        for (int c = tid; c < tail; c += kThreads) {
+            const int64_t col = nvec * VEC + c;
+            const float q[1] = {to_f32(qr[col * a.lq.s_col])};
+            const float p[1] = {to_f32(pr[col * a.lp.s_col])};
+            kl_fold<1>(st, q, p);
+        }
+        kl_group_reduce<32>(st);
+        if (lane == 0) wslots[par][wid] = st;
+        __syncthreads();
+        if (wid == 0) {
+            st = wslots[par][lane & (kKlCtaWarps - 1)];
+            kl_group_reduce<kKlCtaWarps>(st);
+        }
+        // row it - 1: every CTA's state has arrived; the first CTA writes it
+        if (it > 0) {
+            cluster_wait_acquire();
+            finish(prev, par ^ 1);
+        }
+        if (wid == 0 && lane == 0) {
+            st_cluster_v4(dst[par], st.mq, st.sq, st.mp, st.sp);
+            st_cluster_f32(dst[par] + 16, st.w);
+        }
+        cluster_arrive_release();
+        prev = r;
+    }
+    if (it > 0) {
+        cluster_wait_acquire();
+        finish(prev, (it - 1) & 1);
+    }
+}
+
 // The backward needs no reduction: the rows are cut into chunks of
 // kKlChunkVecs vectors, one warp per (row, chunk) unit.
 constexpr int64_t kKlChunkVecs = 1024;
@@ -352,9 +463,55 @@ template <int VEC, bool BWD = false> struct KlShape {
     static constexpr int MINB = VEC == 1 ? 2 : 3;
 };
 
+template <typename T, int VEC, int CL>
+static cudaError_t launch_kl_cluster(const KlPlan& p, const KlArgs& a, cudaStream_t s) {
+    constexpr int U = KlShape<VEC>::U;
+    constexpr int MB = VEC == 1 ? 2 : (VEC == 8 ? 3 : 4);
+    auto kern = k_kl_fwd_cluster<T, VEC, U, CL, MB>;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    cfg.blockDim = dim3(kKlCtaWarps * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = CL;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    // co-resident clusters, cached per device
+    static std::mutex mu;
+    static int cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    int clusters;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        clusters = cached[dev];
+        if (clusters == 0) {
+            cfg.gridDim = dim3(CL * p.sms);
+            const cudaError_t e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+            if (e != cudaSuccess) return e;
+            if (clusters < 1) return cudaErrorInvalidConfiguration;
+            cached[dev] = clusters;
+        }
+    }
+    const int64_t want = a.N < clusters ? a.N : clusters;
+    cfg.gridDim = dim3((unsigned)(want * CL));
+    return cudaLaunchKernelEx(&cfg, kern, a, p.vec_per_cta);
+}
+
 template <typename T, int VEC>
 static cudaError_t kl_fwd_v(const KlPlan& p, const KlArgs& a, cudaStream_t s) {
     constexpr int U = KlShape<VEC>::U, MB = KlShape<VEC>::MINB;
+    if (p.cta && p.cl > 1) {
+        switch (p.cl) {
+            case 2: return launch_kl_cluster<T, VEC, 2>(p, a, s);
+            case 4: return launch_kl_cluster<T, VEC, 4>(p, a, s);
+            case 8: return launch_kl_cluster<T, VEC, 8>(p, a, s);
+        }
+        return cudaErrorInvalidValue;
+    }
     if (p.cta) {
         // four CTAs per SM for 4-byte rows: 592 rows in flight on a 148-SM
         // part, so a batch of a few hundred long rows runs in one wave
