@@ -38,11 +38,9 @@ unsigned int* error_word() {
     return g_err_ptr[dev];
 }
 
-int device_sms(int num_sms) {
-    if (num_sms > 0) return num_sms;
-    const int dev = current_device();
+// SM count of device `dev`, cached; the caller holds g_dev_mutex.
+static int device_sms_locked(int dev) {
     if (dev < 0 || dev >= kMaxDevices) return 148;
-    std::lock_guard<std::mutex> lock(g_dev_mutex);
     if (!g_num_sms[dev]) {
         int n = 0;
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
@@ -50,6 +48,14 @@ int device_sms(int num_sms) {
         g_num_sms[dev] = n;
     }
     return g_num_sms[dev];
+}
+
+int device_sms(int num_sms) {
+    if (num_sms > 0) return num_sms;
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    return device_sms_locked(dev);
 }
 
 // Settings of the testing hook ce_testing_set_wait.
@@ -79,6 +85,33 @@ cudaError_t ensure_smem_limit(const void* kernel, int bytes) {
         cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     g_smem_limits.push_back(SmemLimit{kernel, dev, bytes});
+    return cudaSuccess;
+}
+
+struct ClusterOcc {
+    const void* kernel;
+    int device, clusters;
+};
+static std::vector<ClusterOcc> g_cluster_occ;
+
+cudaError_t max_active_clusters(const void* kernel, const cudaLaunchConfig_t& cfg, int* clusters) {
+    const int dev = current_device();
+    if (dev < 0) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    for (const ClusterOcc& o : g_cluster_occ)
+        if (o.kernel == kernel && o.device == dev) {
+            *clusters = o.clusters;
+            return cudaSuccess;
+        }
+    cudaLaunchConfig_t c = cfg;
+    c.gridDim = dim3((unsigned)(cfg.attrs && cfg.numAttrs ? cfg.attrs[0].val.clusterDim.x : 1) *
+                     (unsigned)device_sms_locked(dev));
+    int n = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kernel, &c);
+    if (e != cudaSuccess) return e;
+    if (n < 1) return cudaErrorInvalidConfiguration;
+    g_cluster_occ.push_back(ClusterOcc{kernel, dev, n});
+    *clusters = n;
     return cudaSuccess;
 }
 

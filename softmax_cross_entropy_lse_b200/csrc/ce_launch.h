@@ -24,6 +24,11 @@ WaitPolicy wait_policy();
 // current device, once per (kernel, device); safe from several threads.
 cudaError_t ensure_smem_limit(const void* kernel, int bytes);
 
+// Clusters of `kernel` that can be resident at once on the current device
+// for the block, cluster and shared-memory shape of `cfg` (its grid is
+// ignored), cached per (kernel, device).
+cudaError_t max_active_clusters(const void* kernel, const cudaLaunchConfig_t& cfg, int* clusters);
+
 // Two-level row addressing: row r starts at (r / inner) * s_outer +
 // (r % inner) * s_inner elements, column j a further j * s_col on.
 struct Layout {

@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
     __shared__ OnlineState wslot[2][kSmWarps];
     // CTA states of the cluster, pushed by their owners: [row parity][source
     // rank][two 16-byte words], completed on xbar[row parity]
-    __shared__ __align__(16) uint4 xslot[2][4][2];
+    __shared__ __align__(16) uint4 xslot[2][CL][2];
     __shared__ __align__(8) uint64_t xbar[2];
     __shared__ int abort_flag;
 

@@ -333,7 +333,10 @@ __global__ void __launch_bounds__(kCtaThreads, kCtaMinBlocks) k_fwd_cta(FwdArgs 
 // full with 1-D bulk copies issued kRingStages chunks ahead (across unit
 // boundaries), and the lanes fold each chunk straight from shared memory. The
 // bytes in flight per SM are set by the rings (up to 192 KB), not by the
-// registers of the folding threads. Chunk c of a unit belongs to warp
+// registers of the folding threads. Four warps with 8 KB stages (three CTAs,
+// twelve warps per SM) measured ahead of eight warps with 4 KB stages: the
+// per-chunk wait, fence and refill and the per-unit exchange are paid over
+// twice the elements, and each lane folds 64 values per part. Chunk c of a unit belongs to warp
 // c % kRingWarps; the warps of a unit meet once, in one exchange of states:
 // each warp writes its state to a slot and arrives on a named barrier without
 // waiting, and only the unit's finaliser (a role that rotates over the warps)
@@ -343,10 +346,10 @@ __global__ void __launch_bounds__(kCtaThreads, kCtaMinBlocks) k_fwd_cta(FwdArgs 
 // later (so no slot is rewritten before it is read: the race of "One barrier
 // short" cannot occur), and the warps of a CTA stay within two units of each
 // other, streaming neighbouring parts of the same rows.
-constexpr int kRingWarps = 8;
+constexpr int kRingWarps = 4;
 constexpr int kRingStages = 2;
-constexpr int kRingVecs = 256;  // 4 KB per stage
-constexpr int kRingPart = 128;  // vectors folded at a time (4 per lane)
+constexpr int kRingVecs = 512;  // 8 KB per stage
+constexpr int kRingPart = 256;  // vectors folded at a time (8 per lane)
 constexpr size_t kRingSmem = (size_t)kRingWarps * kRingStages * kRingVecs * 16;
 static_assert((kRingStages & (kRingStages - 1)) == 0 && (kRingWarps & (kRingWarps - 1)) == 0,
               "stage and warp counts are powers of two");
@@ -480,7 +483,7 @@ __global__ void __launch_bounds__(kRingWarps * 32, 3) k_fwd_ring(FwdArgs a) {
             if (!dead) {
                 const int64_t left = ru.nv - (int64_t)j * kRingVecs;
                 const int nvc = (int)(left < kRingVecs ? left : kRingVecs);
-                // the chunk is folded in parts of kRingPart vectors (4 per lane)
+                // the chunk is folded in parts of kRingPart vectors
 #pragma unroll 1
                 for (int h = 0; h < kRingVecs / kRingPart && h * kRingPart < nvc; ++h) {
                     const uint4* buf =
