@@ -8,13 +8,17 @@ backward of Z = H W^T without storing Z). Default workload: 1,048,576 rows x
 128 classes, fp32 logits ~N(0,1), 10% of targets at ignore_index=-100,
 label smoothing 0.1.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2] [--also LIST]
     python bench.py --impl reference ...   (the float64 CPU oracle, timed)
 
-Prints one JSON line (rank 0). For N > 1 it is launched with torchrun, one
-rank per GPU; every rank processes its own batch (rows are independent, no
-data-path collective), the device time is the max over ranks and the value
-is the bytes of all ranks over that time.
+Prints one JSON line (rank 0). With the default headline (c2) the line also
+carries, under "workloads", the same measurements for every other workload
+(c1, c3a, c3b, c4a, c4b, c5, soft, kl), each with its rates, roofline,
+clocks and end-to-end rate; --also chooses them ("none" for the headline
+alone). For N > 1 it is launched with torchrun, one rank per GPU; every rank
+processes its own batch (rows are independent, no data-path collective), the
+device time is the max over ranks and the value is the bytes of all ranks over
+that time.
 """
 from __future__ import annotations
 

@@ -13,7 +13,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libce_b200.so")
 SOURCES = ["ce_api.cu", "ce_rows_fwd.cu", "ce_rows_bwd.cu", "ce_rows_fused.cu",
-           "ce_rows_fused_smem.cu", "ce_rows_soft.cu", "ce_rows_kl.cu",
+           "ce_rows_fused_slices.cu", "ce_rows_soft.cu", "ce_rows_kl.cu",
            "ce_linear.cu", "ce_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",

@@ -731,24 +731,34 @@ ce_status ce_forward_backward(const void* logits, ce_dtype dt, ce_layout lg, int
     int G = 1;
     while (G < 32 && nvec > (int64_t)kU * G) G *= 2;
     const int sms = device_sms(0);
-    // rows beyond one warp's registers: held in shared memory by a cluster of
-    // the fewest CTAs whose slices fit (needs 16-byte rows, and enough rows
-    // to give every SM a CTA); else a forward, then the VJP
-    SmemRowPlan sp{};
+    // rows beyond one warp's registers: one slice per CTA, held in shared
+    // memory when the row fits one CTA's 112 KB, else re-read through L2 by a
+    // cluster of the fewest CTAs (up to 8) whose slices are at most 128 KB.
+    // Both need 16-byte rows, and enough rows to give every SM a CTA; else a
+    // forward, then the VJP.
+    SliceRowPlan sp{};
     if (nvec > (int64_t)kU * G && vec_ok) {
-        // clusters of up to 4 CTAs: rows that need 8 (over 448 KB, e.g. 151,936
-        // fp32) measured slower than the forward followed by the VJP
-        for (int cl = 1; cl <= 4; cl *= 2) {
-            const int64_t per = (nvec + cl - 1) / cl;
-            const int64_t nch = (per + 127) / 128;
-            if (nch <= kSmemRowMaxChunks) {
-                if (N * cl >= sms) {
-                    sp.cl = cl;
-                    sp.nch = (int)nch;
-                    sp.vec_per_cta = per;
-                    sp.sms = sms;
+        if (nvec <= (int64_t)kSliceSmemMaxChunks * 128) {
+            if (N >= sms) {
+                sp.cl = 1;
+                sp.nch = (int)((nvec + 127) / 128);
+                sp.vec_per_cta = nvec;
+                sp.sms = sms;
+                sp.l2 = 0;
+            }
+        } else {
+            for (int cl = 1; cl <= 8; cl *= 2) {
+                const int64_t per = (nvec + cl - 1) / cl;
+                if (per * 16 <= kSliceL2MaxBytes) {
+                    if (N * cl >= sms) {
+                        sp.cl = cl;
+                        sp.nch = (int)((per + 127) / 128);
+                        sp.vec_per_cta = per;
+                        sp.sms = sms;
+                        sp.l2 = 1;
+                    }
+                    break;
                 }
-                break;
             }
         }
     }
@@ -823,7 +833,7 @@ ce_status ce_forward_backward(const void* logits, ce_dtype dt, ce_layout lg, int
     a.dz = dlogits;
     a.ld = D;
     cudaError_t e = sp.cl > 0
-                        ? launch_fused_smem(sp, a, (int)dt, (int)ddt, static_cast<cudaStream_t>(cuda_stream))
+                        ? launch_fused_slices(sp, a, (int)dt, (int)ddt, static_cast<cudaStream_t>(cuda_stream))
                         : launch_fused(p, a, (int)dt, (int)ddt, static_cast<cudaStream_t>(cuda_stream));
     return e == cudaSuccess ? CE_OK : CE_ECUDA;
 }

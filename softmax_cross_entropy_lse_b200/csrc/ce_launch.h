@@ -126,20 +126,25 @@ struct FusedPlan {
 cudaError_t launch_fused(const FusedPlan& p, const FusedArgs& a, int dt_in, int dt_out,
                          cudaStream_t s);
 
-// ---- fused forward + backward (rows held in shared memory) -----------------
+// ---- fused forward + backward of long rows, one slice per CTA ---------------
 // A row is split over a cluster of `cl` CTAs, vec_per_cta 16-byte vectors
-// each, held in nch 2 KB chunks of shared memory.
-constexpr int kSmemRowMaxChunks = 56;  // 112 KB per CTA: two CTAs per SM
+// (nch 2 KB chunks) each. The slice is held in shared memory (l2 = 0; one CTA
+// per row, up to kSliceSmemMaxChunks chunks), or read twice from global
+// memory with the second read served by L1/L2 (l2 = 1; slices up to
+// kSliceL2MaxBytes, clusters of 1 to 8).
+constexpr int kSliceSmemMaxChunks = 56;           // 112 KB per CTA: two CTAs per SM
+constexpr int64_t kSliceL2MaxBytes = 128 * 1024;  // 148 SMs x 4 CTAs: 76 MB of L2
 
-struct SmemRowPlan {
+struct SliceRowPlan {
     int cl;
     int nch;
     int64_t vec_per_cta;
     int sms;
+    int l2;
 };
 
-cudaError_t launch_fused_smem(const SmemRowPlan& p, const FusedArgs& a, int dt_in, int dt_out,
-                              cudaStream_t s);
+cudaError_t launch_fused_slices(const SliceRowPlan& p, const FusedArgs& a, int dt_in, int dt_out,
+                                cudaStream_t s);
 
 // ---- probability (soft) targets ---------------------------------------------
 struct SoftArgs {

@@ -1,34 +1,41 @@
-// Fused forward + VJP for rows held in shared memory (rows too long for one
-// warp's registers, up to 4 x 112 KB).
+// Fused forward + VJP for rows too long for one warp's registers.
 //
 // When g is known before the forward runs, the gradient
 //     dz_j = g (exp(z_j - lse) - (1 - eps)[j = y] - eps/V)
-// needs nothing but the row and its lse, so the row is read from HBM once:
-// it is copied into shared memory, folded into the online (max, scaled sum)
-// state of Ineshin, "A fused linear cross-entropy forward kernel for Apple
-// GPUs", section 1, reduced, and then read a second time from shared memory
-// to form dz. HBM traffic is 2 V e per row instead of the 3 V e of a forward
-// followed by a VJP that re-reads the logits (the backward regenerates from
-// the saved lse, section 1 of the same page).
+// needs nothing but the row and its lse, so the row crosses HBM once: it is
+// folded into the online (max, scaled sum) state of Ineshin, "A fused linear
+// cross-entropy forward kernel for Apple GPUs", section 1, reduced, and then
+// read a second time, from on-chip memory, to form dz. HBM traffic is 2 V e
+// per row instead of the 3 V e of a forward followed by a VJP that re-reads
+// the logits (the backward regenerates from the saved lse, section 1 of the
+// same page).
 //
-// A row longer than one CTA's share of shared memory is split across a
-// thread-block cluster of CL CTAs (CL = 1, 2, 4); CTA k holds vectors
-// [k S, (k+1) S) of the row. Each CTA reduces its slice and pushes its state
-// into the shared memory of every other CTA of the cluster (st.async,
-// completed on the receiver's mbarrier, so no cluster-wide barrier or fence
-// runs per row); every CTA merges the CL states in rank order, so all of them
-// derive the same lse bits.
-//
-// Within a CTA, 8 warps own the 2 KB chunks of the slice round-robin (chunk c
-// belongs to warp c % 8). A warp's lane 0 copies its chunks in with 1-D bulk
-// copies (TMA engine), the warp folds them as they land, and once its
-// gradient pass over them is done it refills them with the next row's bytes:
-// no CTA-wide barrier guards the buffers, and the next row streams in while
-// the other warps are still differentiating this one. The warp and CTA states of row
-// i use exchange slots of parity i & 1, so no slot is rewritten before every
-// reader has passed the next barrier (the race of Suryavanshi, "One barrier
-// short", cannot occur). Every wait is bounded; on expiry the kernel raises
-// error bit 2, stops issuing copies, drains those in flight and returns.
+// A row is cut into slices, one per CTA of a thread-block cluster of CL CTAs;
+// CTA k holds vectors [k S, (k+1) S). Within a CTA, 8 warps own the 2 KB
+// chunks of the slice round-robin (chunk c belongs to warp c % 8). Two ways to
+// keep the slice on chip between its two reads:
+//  * shared memory (rows up to 112 KB, one CTA per row): a warp's lane 0
+//    copies its chunks in with 1-D bulk copies (TMA engine), the warp folds
+//    them as they land, and once its gradient pass over them is done it
+//    refills them with the next row's bytes: no CTA-wide barrier guards the
+//    buffers, and the next row streams in while the other warps are still
+//    differentiating this one. Two or three CTAs per SM.
+//  * L2 (longer rows; slices of at most 128 KB): the slice is read from
+//    global memory twice, and the second read hits the L1 or the L2, where
+//    the first left it (at four CTAs per SM the slices in flight take at most
+//    148 x 4 x 128 KB = 76 MB of the 126 MB L2). No shared memory holds row
+//    data, so four CTAs fit per SM instead of two and cover one another's
+//    waits on the cluster exchange; on 2048 x 151,936 bf16 rows this ran 11 %
+//    ahead of 76 KB slices in shared memory.
+// Each CTA reduces its slice and pushes its state into the shared memory of
+// every other CTA of the cluster (st.async, completed on the receiver's
+// mbarrier, so no cluster-wide barrier or fence runs per row); every CTA
+// merges the CL states in rank order, so all of them derive the same lse
+// bits. The warp and CTA states of row i use exchange slots of parity i & 1,
+// so no slot is rewritten before every reader has passed the next barrier
+// (the race of Suryavanshi, "One barrier short", cannot occur). Every wait is
+// bounded; on expiry the kernel raises error bit 2, stops issuing copies,
+// drains those in flight and returns.
 #include "ce_device.cuh"
 #include "ce_launch.h"
 #include "ce_sm100.cuh"
@@ -39,7 +46,7 @@ namespace ceb {
 
 constexpr int kSmWarps = 8;
 constexpr int kSmChunkVecs = 128;  // 16-byte vectors per 2 KB chunk
-constexpr int kSmMaxChunks = kSmemRowMaxChunks;
+constexpr int kSmMaxChunks = kSliceSmemMaxChunks;
 static_assert(kSmMaxChunks <= 8 * 32, "per-warp chunk masks are 32 bits");
 
 // Pushes 16 bytes into the shared memory of another CTA of the cluster
@@ -54,22 +61,19 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, const uint4& v
         : "memory");
 }
 
-// Folds one chunk. 16-bit rows without argmax or label smoothing fold every
-// chunk after a lane's first against the lane's reference max (ref).
+// Folds one chunk held as words w (lane's vectors q * 32 + lane, q < 4).
+// 16-bit rows without argmax or label smoothing fold every chunk after a
+// lane's first against the lane's reference max (ref).
 template <typename TI, bool ARGMAX, bool WITH_T>
-__device__ __forceinline__ void fold_chunk(OnlineState& st, FoldRef& ref, const uint4* buf, int nvc,
-                                           int lane, int64_t col_vec0) {
+__device__ __forceinline__ void fold_words(OnlineState& st, FoldRef& ref,
+                                           const uint4 (&w)[kSmChunkVecs / 32], int nvc, int lane,
+                                           int64_t col_vec0) {
     constexpr int VEC = ElemTraits<TI>::kVec;
     constexpr int kPerLane = kSmChunkVecs / 32;
-    if constexpr (sizeof(TI) == 2 && !ARGMAX) {
-        uint4 w[kPerLane];
-        bool ok[kPerLane];
+    bool ok[kPerLane];
 #pragma unroll
-        for (int q = 0; q < kPerLane; ++q) {
-            const int vi = q * 32 + lane;
-            ok[q] = vi < nvc;
-            if (ok[q]) w[q] = buf[vi];
-        }
+    for (int q = 0; q < kPerLane; ++q) ok[q] = q * 32 + lane < nvc;
+    if constexpr (sizeof(TI) == 2 && !ARGMAX) {
         if (nvc == kSmChunkVecs) {
             bool done = false;
             if constexpr (!WITH_T) {
@@ -85,14 +89,11 @@ __device__ __forceinline__ void fold_chunk(OnlineState& st, FoldRef& ref, const 
         }
     } else {
         float v[kPerLane][VEC];
-        bool ok[kPerLane];
         int c0[kPerLane];
 #pragma unroll
         for (int q = 0; q < kPerLane; ++q) {
-            const int vi = q * 32 + lane;
-            ok[q] = vi < nvc;
-            c0[q] = (int)((col_vec0 + vi) * VEC);
-            if (ok[q]) unpack_words<TI>(buf[vi], v[q]);
+            c0[q] = (int)((col_vec0 + q * 32 + lane) * VEC);
+            if (ok[q]) unpack_words<TI>(w[q], v[q]);
         }
         if (nvc == kSmChunkVecs) {
             fold_vecs<kPerLane, VEC, false>(st, v, ok);
@@ -104,54 +105,113 @@ __device__ __forceinline__ void fold_chunk(OnlineState& st, FoldRef& ref, const 
     }
 }
 
-// dz of one chunk from its shared-memory copy. `cst` is 0 for ordinary rows;
-// ignored rows write 0 and rows with a bad target NaN (cst_mode 1 / 2).
+// Loads a lane's words of one chunk (vectors q * 32 + lane below nvc) from
+// shared or global memory; LAST marks the last read of global data.
+template <bool LAST = false>
+__device__ __forceinline__ void load_chunk(uint4 (&w)[kSmChunkVecs / 32], const uint4* buf, int nvc,
+                                           int lane) {
+#pragma unroll
+    for (int q = 0; q < kSmChunkVecs / 32; ++q) {
+        const int vi = q * 32 + lane;
+        if (vi < nvc) w[q] = LAST ? __ldcs(buf + vi) : buf[vi];
+    }
+}
+
+template <typename TI, bool ARGMAX, bool WITH_T>
+__device__ __forceinline__ void fold_chunk(OnlineState& st, FoldRef& ref, const uint4* buf, int nvc,
+                                           int lane, int64_t col_vec0) {
+    uint4 w[kSmChunkVecs / 32];
+    load_chunk(w, buf, nvc, lane);
+    fold_words<TI, ARGMAX, WITH_T>(st, ref, w, nvc, lane, col_vec0);
+}
+
+// dz of the vectors q * 32 + lane of one chunk (all of them when FULL),
+// from the words w; TGT: the target column lies in this chunk, dyc columns
+// after its start.
+template <typename TI, typename TO, bool FULL, bool TGT>
+__device__ __forceinline__ void grad_words_k(const uint4 (&w)[kSmChunkVecs / 32], int nvc, int lane,
+                                             TO* dchunk, float hi, float c_lo, float g, float c_eps,
+                                             float c_tgt, int dyc) {
+    constexpr int VEC = ElemTraits<TI>::kVec;
+    const float2 nhi = make_float2(-hi, -hi), l2 = make_float2(kLog2e, kLog2e);
+    const float2 nclo = make_float2(-c_lo, -c_lo), g2 = make_float2(g, g);
+    const float2 nce = make_float2(-c_eps, -c_eps);
+#pragma unroll
+    for (int q = 0; q < kSmChunkVecs / 32; ++q) {
+        const int vi = q * 32 + lane;
+        if (!FULL && vi >= nvc) continue;
+        float x[VEC], o[VEC];
+        unpack_words<TI>(w[q], x);
+#pragma unroll
+        for (int e = 0; e < VEC; e += 2) {
+            const float2 d = __fadd2_rn(make_float2(x[e], x[e + 1]), nhi);
+            const float2 arg = __ffma2_rn(d, l2, nclo);
+            const float2 p = make_float2(ex2(arg.x), ex2(arg.y));
+            const float2 r = __ffma2_rn(g2, p, nce);
+            o[e] = r.x;
+            o[e + 1] = r.y;
+        }
+        if constexpr (TGT) {
+            const int dy = dyc - vi * VEC;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e)
+                if (dy == e) o[e] -= c_tgt;
+        }
+        store_vec<TO, VEC>(dchunk, (int64_t)vi * VEC, 1, o);
+    }
+}
+
+// dz of one chunk. `cst_mode` is 0 for ordinary rows; ignored rows write 0
+// and rows with a bad target NaN (cst_mode 1 / 2). The chunk that holds the
+// target (one per row) takes a separate, warp-uniform branch, so the others
+// pay nothing for the target's term.
+template <typename TI, typename TO>
+__device__ __forceinline__ void grad_words(const uint4 (&w)[kSmChunkVecs / 32], int nvc, int lane,
+                                           int64_t col_vec0, TO* drow, float hi, float c_lo, float g,
+                                           float c_eps, float c_tgt, int64_t yc, int cst_mode) {
+    constexpr int VEC = ElemTraits<TI>::kVec;
+    const int64_t col_chunk = col_vec0 * VEC;
+    TO* dchunk = drow + col_chunk;
+    if (cst_mode != 0) {
+        const float fill = cst_mode == 2 ? __int_as_float(0x7fc00000) : 0.f;
+        float o[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) o[e] = fill;
+#pragma unroll
+        for (int q = 0; q < kSmChunkVecs / 32; ++q) {
+            const int vi = q * 32 + lane;
+            if (vi < nvc) store_vec<TO, VEC>(dchunk, (int64_t)vi * VEC, 1, o);
+        }
+    } else if (yc >= col_chunk && yc < col_chunk + (int64_t)nvc * VEC) {
+        grad_words_k<TI, TO, false, true>(w, nvc, lane, dchunk, hi, c_lo, g, c_eps, c_tgt,
+                                          (int)(yc - col_chunk));
+    } else if (nvc == kSmChunkVecs) {
+        grad_words_k<TI, TO, true, false>(w, nvc, lane, dchunk, hi, c_lo, g, c_eps, c_tgt, 0);
+    } else {
+        grad_words_k<TI, TO, false, false>(w, nvc, lane, dchunk, hi, c_lo, g, c_eps, c_tgt, 0);
+    }
+}
+
 template <typename TI, typename TO>
 __device__ __forceinline__ void grad_chunk(const uint4* buf, int nvc, int lane, int64_t col_vec0,
                                            TO* drow, float hi, float c_lo, float g, float c_eps,
                                            float c_tgt, int64_t yc, int cst_mode) {
-    constexpr int VEC = ElemTraits<TI>::kVec;
-    constexpr int kPerLane = kSmChunkVecs / 32;
-    const int64_t col_chunk = col_vec0 * VEC;
-    const bool has_y = yc >= col_chunk && yc < col_chunk + (int64_t)nvc * VEC;
-    const float2 nhi = make_float2(-hi, -hi), l2 = make_float2(kLog2e, kLog2e);
-    const float2 nclo = make_float2(-c_lo, -c_lo), g2 = make_float2(g, g);
-    const float2 nce = make_float2(-c_eps, -c_eps);
-    const float fill = cst_mode == 2 ? __int_as_float(0x7fc00000) : 0.f;
-#pragma unroll
-    for (int q = 0; q < kPerLane; ++q) {
-        const int vi = q * 32 + lane;
-        if (vi >= nvc) continue;
-        const int64_t col0 = (col_vec0 + vi) * VEC;
-        float o[VEC];
-        if (cst_mode != 0) {
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) o[e] = fill;
-        } else {
-            float x[VEC];
-            unpack_words<TI>(buf[vi], x);
-#pragma unroll
-            for (int e = 0; e < VEC; e += 2) {
-                const float2 d = __fadd2_rn(make_float2(x[e], x[e + 1]), nhi);
-                const float2 arg = __ffma2_rn(d, l2, nclo);
-                const float2 p = make_float2(ex2(arg.x), ex2(arg.y));
-                const float2 r = __ffma2_rn(g2, p, nce);
-                o[e] = r.x;
-                o[e + 1] = r.y;
-            }
-            if (has_y) {
-                const int64_t dy = yc - col0;
-#pragma unroll
-                for (int e = 0; e < VEC; ++e)
-                    if (dy == e) o[e] -= c_tgt;
-            }
-        }
-        store_vec<TO, VEC>(drow, col0, 1, o);
-    }
+    uint4 w[kSmChunkVecs / 32];
+    if (cst_mode == 0) load_chunk(w, buf, nvc, lane);
+    grad_words<TI, TO>(w, nvc, lane, col_vec0, drow, hi, c_lo, g, c_eps, c_tgt, yc, cst_mode);
 }
 
-template <typename TI, typename TO, int CL, bool ARGMAX, bool WITH_T>
-__global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, SmemRowPlan sp) {
+// Occupancy targets: up to three CTAs per SM hold their slices in shared
+// memory (two at 112 KB); slices re-read through L2 leave room for four
+// (three with argmax, whose extra state would spill at 64 registers a thread).
+template <bool ARGMAX, bool GL>
+struct SliceShape {
+    static constexpr int kMinBlocks = GL ? (ARGMAX ? 3 : 4) : 3;
+};
+
+template <typename TI, typename TO, int CL, bool ARGMAX, bool WITH_T, bool GL>
+__global__ void __launch_bounds__(kSmWarps * 32, (SliceShape<ARGMAX, GL>::kMinBlocks))
+    k_fwdbwd_slices(FusedArgs fa, SliceRowPlan sp) {
     using namespace sm100;
     constexpr int VEC = ElemTraits<TI>::kVec;
     const FwdArgs& a = fa.f;
@@ -180,7 +240,7 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
     const RowOut out{a.loss, a.lse, a.lse_lo, a.argmax, a.err};
     const float inv_v = 1.f / (float)a.V;
 
-    if (lane == 0)
+    if (!GL && lane == 0)
         for (int c = wid; c < nch; c += kSmWarps) mbar_init(smem_u32(&full_bar[c]), 1);
     if (tid == 0) {
         abort_flag = 0;
@@ -205,7 +265,7 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
 
     // bit i of the masks: this warp's i-th chunk (c = wid + 8 i)
     uint32_t pend = 0, phase = 0;
-    if (cid < a.N) {
+    if (!GL && cid < a.N) {
         for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps) {
             if (lane == 0) issue(cid, c);
             pend |= 1u << i;
@@ -226,11 +286,21 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
         float zy = 0.f;
         if (rank == 0 && tid == 0 && yc >= 0) zy = to_f32(row[yc]);
 
-        // ---- forward: fold the slice as its chunks land
+        // ---- forward: fold the slice (from global memory, or from shared
+        // memory as its chunks land)
         OnlineState st = empty_state();
         FoldRef ref;
         ref.ok = false;
-        for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps) {
+        const uint4* grow = reinterpret_cast<const uint4*>(row) + v0;
+        if constexpr (GL) {
+            for (int c = wid; c < nch; c += kSmWarps) {
+                uint4 w[kSmChunkVecs / 32];
+                load_chunk(w, grow + (int64_t)c * kSmChunkVecs, chunk_vecs(c), lane);
+                fold_words<TI, ARGMAX, WITH_T>(st, ref, w, chunk_vecs(c), lane,
+                                               v0 + (int64_t)c * kSmChunkVecs);
+            }
+        }
+        for (int i = 0, c = wid; !GL && c < nch; ++i, c += kSmWarps) {
             if (!dead) {
                 if (mbar_wait(smem_u32(&full_bar[c]), (phase >> i) & 1u, &abort_flag)) {
                     phase ^= 1u << i;
@@ -292,22 +362,32 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
         }
         if (rank == 0 && tid == 0) finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);
 
-        // ---- backward from the same shared-memory copy
+        // ---- backward from the on-chip copy
         float L, hi, lo;
         lse_pair(st, L, hi, lo);
         const float c_lo = lo * kLog2e, c_eps = g * a.eps * inv_v, c_tgt = g * (1.f - a.eps);
         const int cst_mode = bad ? 2 : (ign ? 1 : 0);
         const int64_t rn = r + ncl;
-        for (int c = wid; c < nch; c += kSmWarps) {
+        if constexpr (GL) {
+            // second read of the slice: L1 or L2 hits, the last use
+            for (int c = wid; !dead && c < nch; c += kSmWarps) {
+                uint4 w[kSmChunkVecs / 32];
+                if (cst_mode == 0)
+                    load_chunk<true>(w, grow + (int64_t)c * kSmChunkVecs, chunk_vecs(c), lane);
+                grad_words<TI, TO>(w, chunk_vecs(c), lane, v0 + (int64_t)c * kSmChunkVecs, drow, hi,
+                                   c_lo, g, c_eps, c_tgt, yc, cst_mode);
+            }
+        }
+        for (int c = wid; !GL && c < nch; c += kSmWarps) {
             if (!dead)
                 grad_chunk<TI, TO>(chunk_buf(c), chunk_vecs(c), lane, v0 + (int64_t)c * kSmChunkVecs,
                                    drow, hi, c_lo, g, c_eps, c_tgt, yc, cst_mode);
         }
         // this warp's chunks are read: refill them with the next row's bytes
         // (one proxy fence for all of them)
-        fence_proxy_async_smem();
+        if constexpr (!GL) fence_proxy_async_smem();
         __syncwarp();
-        if (rn < a.N && !dead) {
+        if (!GL && rn < a.N && !dead) {
             for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps) {
                 if (lane == 0) issue(rn, c);
                 pend |= 1u << i;
@@ -334,7 +414,7 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
         if (lane == 0) atomicOr(a.err, kErrTimeout);
         // let every copy this warp started land before the CTA exits
         volatile int never = 0;
-        for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps)
+        for (int i = 0, c = wid; !GL && c < nch; ++i, c += kSmWarps)
             if ((pend >> i) & 1u) mbar_wait(smem_u32(&full_bar[c]), (phase >> i) & 1u, &never);
     }
     // no CTA leaves while a peer may still push into its slots
@@ -342,14 +422,14 @@ __global__ void __launch_bounds__(kSmWarps * 32, 3) k_fwdbwd_smem(FusedArgs fa, 
 }
 
 // ---------------------------------------------------------------------------
-template <typename TI, typename TO, int CL, bool ARGMAX, bool WITH_T>
-static cudaError_t launch_smem_k(const SmemRowPlan& sp, const FusedArgs& a, cudaStream_t s) {
-    auto kern = k_fwdbwd_smem<TI, TO, CL, ARGMAX, WITH_T>;
-    {
+template <typename TI, typename TO, int CL, bool ARGMAX, bool WITH_T, bool GL>
+static cudaError_t launch_slices_k(const SliceRowPlan& sp, const FusedArgs& a, cudaStream_t s) {
+    auto kern = k_fwdbwd_slices<TI, TO, CL, ARGMAX, WITH_T, GL>;
+    if constexpr (!GL) {
         cudaError_t e = ensure_smem_limit((const void*)kern, kSmMaxChunks * 2048);
         if (e != cudaSuccess) return e;
     }
-    const size_t smem = (size_t)sp.nch * 2048;
+    const size_t smem = GL ? 0 : (size_t)sp.nch * 2048;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
     cfg.blockDim = dim3(kSmWarps * 32);
@@ -387,30 +467,34 @@ static cudaError_t launch_smem_k(const SmemRowPlan& sp, const FusedArgs& a, cuda
     return cudaLaunchKernelEx(&cfg, kern, a, sp);
 }
 
+// Shared-memory slices run one CTA per row; L2 slices take clusters of 1 to 8.
 template <typename TI, typename TO, bool ARGMAX, bool WITH_T>
-static cudaError_t launch_smem_cl(const SmemRowPlan& sp, const FusedArgs& a, cudaStream_t s) {
+static cudaError_t launch_slices_cl(const SliceRowPlan& sp, const FusedArgs& a, cudaStream_t s) {
+    if (!sp.l2) return sp.cl == 1 ? launch_slices_k<TI, TO, 1, ARGMAX, WITH_T, false>(sp, a, s)
+                                  : cudaErrorInvalidValue;
     switch (sp.cl) {
-        case 1: return launch_smem_k<TI, TO, 1, ARGMAX, WITH_T>(sp, a, s);
-        case 2: return launch_smem_k<TI, TO, 2, ARGMAX, WITH_T>(sp, a, s);
-        case 4: return launch_smem_k<TI, TO, 4, ARGMAX, WITH_T>(sp, a, s);
+        case 1: return launch_slices_k<TI, TO, 1, ARGMAX, WITH_T, true>(sp, a, s);
+        case 2: return launch_slices_k<TI, TO, 2, ARGMAX, WITH_T, true>(sp, a, s);
+        case 4: return launch_slices_k<TI, TO, 4, ARGMAX, WITH_T, true>(sp, a, s);
+        case 8: return launch_slices_k<TI, TO, 8, ARGMAX, WITH_T, true>(sp, a, s);
     }
     return cudaErrorInvalidValue;
 }
 
 template <typename TI, typename TO>
-static cudaError_t launch_smem_t(const SmemRowPlan& sp, const FusedArgs& a, cudaStream_t s) {
+static cudaError_t launch_slices_t(const SliceRowPlan& sp, const FusedArgs& a, cudaStream_t s) {
     const bool am = a.f.argmax != nullptr, t = a.f.eps != 0.f;
-    if (am) return t ? launch_smem_cl<TI, TO, true, true>(sp, a, s) : launch_smem_cl<TI, TO, true, false>(sp, a, s);
-    return t ? launch_smem_cl<TI, TO, false, true>(sp, a, s) : launch_smem_cl<TI, TO, false, false>(sp, a, s);
+    if (am) return t ? launch_slices_cl<TI, TO, true, true>(sp, a, s) : launch_slices_cl<TI, TO, true, false>(sp, a, s);
+    return t ? launch_slices_cl<TI, TO, false, true>(sp, a, s) : launch_slices_cl<TI, TO, false, false>(sp, a, s);
 }
 
-cudaError_t launch_fused_smem(const SmemRowPlan& sp, const FusedArgs& a, int dt_in, int dt_out,
-                              cudaStream_t s) {
-    if (dt_in == 0 && dt_out == 0) return launch_smem_t<float, float>(sp, a, s);
-    if (dt_in == 1 && dt_out == 1) return launch_smem_t<__nv_bfloat16, __nv_bfloat16>(sp, a, s);
-    if (dt_in == 1 && dt_out == 0) return launch_smem_t<__nv_bfloat16, float>(sp, a, s);
-    if (dt_in == 2 && dt_out == 2) return launch_smem_t<__half, __half>(sp, a, s);
-    if (dt_in == 2 && dt_out == 0) return launch_smem_t<__half, float>(sp, a, s);
+cudaError_t launch_fused_slices(const SliceRowPlan& sp, const FusedArgs& a, int dt_in, int dt_out,
+                                cudaStream_t s) {
+    if (dt_in == 0 && dt_out == 0) return launch_slices_t<float, float>(sp, a, s);
+    if (dt_in == 1 && dt_out == 1) return launch_slices_t<__nv_bfloat16, __nv_bfloat16>(sp, a, s);
+    if (dt_in == 1 && dt_out == 0) return launch_slices_t<__nv_bfloat16, float>(sp, a, s);
+    if (dt_in == 2 && dt_out == 2) return launch_slices_t<__half, __half>(sp, a, s);
+    if (dt_in == 2 && dt_out == 0) return launch_slices_t<__half, float>(sp, a, s);
     return cudaErrorInvalidValue;
 }
 

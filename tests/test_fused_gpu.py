@@ -145,14 +145,18 @@ def _padded(N, V, pad, dtype, seed, std=2.0, ignore_frac=0.1):
 
 
 @pytest.mark.parametrize("V,N,dt", [
-    (2048, 400, "bf16"),       # one CTA, 2 chunks
-    (32000, 600, "bf16"),      # one CTA, the 8192 x 32000 row shape
-    (33000, 300, "f16"),       # one CTA, partial last chunk
-    (100000, 200, "bf16"),     # cluster of 2
-    (151936, 160, "bf16"),     # cluster of 4, the 2048 x 151,936 row shape
-    (20000, 300, "f32"),       # one CTA, fp32
-    (100000, 80, "f32"),       # cluster of 4, fp32
-    (151936, 40, "f32"),       # 608 KB rows: the forward, then the VJP
+    (2048, 400, "bf16"),       # shared memory, one CTA, 2 chunks
+    (32000, 600, "bf16"),      # shared memory, the 8192 x 32000 row shape
+    (33000, 300, "f16"),       # shared memory, partial last chunk
+    (57344, 300, "bf16"),      # shared memory, the largest row (56 chunks, 112 KB)
+    (57352, 300, "bf16"),      # one vector more: an L2 slice, cluster of 1
+    (100000, 200, "bf16"),     # L2 slices, cluster of 2
+    (151936, 160, "bf16"),     # L2 slices, cluster of 4, the 2048 x 151,936 row shape
+    (20000, 300, "f32"),       # shared memory, fp32
+    (100000, 80, "f32"),       # L2 slices, cluster of 4, fp32
+    (151936, 40, "f32"),       # L2 slices, cluster of 8 (608 KB rows)
+    (151936, 30, "bf16"),      # too few rows for every SM: the forward, then the VJP
+    (600000, 12, "bf16"),      # beyond 8 slices of 128 KB: the forward, then the VJP
 ])
 def test_smem_rows_vs_oracle(orc, V, N, dt):
     z, z32, y = wl.rows(N, V, dt, seed=V % 997 + N, std=2.0, ignore_frac=0.1)
@@ -176,10 +180,12 @@ def test_smem_rows_vs_oracle(orc, V, N, dt):
 
 
 @pytest.mark.parametrize("out", ["bf16", "f32"])
-def test_smem_rows_ragged_tail_views(orc, out):
-    """V = 32005 (5 columns past the last 16-byte vector), rows of a padded
-    buffer; dlogits is a padded view too, in bf16 or float."""
-    N, V, pad = 300, 32005, 3
+@pytest.mark.parametrize("V", [32005, 100005])
+def test_smem_rows_ragged_tail_views(orc, out, V):
+    """V = 32005 (shared memory) and 100005 (L2 slices, cluster of 2): 5
+    columns past the last 16-byte vector, rows of a padded buffer; dlogits is
+    a padded view too, in bf16 or float."""
+    N, pad = 300, 3
     z, z32, y = _padded(N, V, pad, "bf16", seed=5)
     zt = upload(z, "bf16")[:, :V]
     yt = upload(y)
@@ -194,8 +200,8 @@ def test_smem_rows_ragged_tail_views(orc, out):
 
 
 def test_long_rows_strided_3d_view(orc):
-    """The (B, L, V) view x[:, :-1] at V = 151,936 fp32 (rows of 607,744 bytes,
-    beyond four CTAs' shared memory: the forward, then the VJP), targets t[:, 1:]."""
+    """The (B, L, V) view x[:, :-1] at V = 151,936 fp32 (rows of 607,744 bytes:
+    L2 slices, cluster of 8), targets t[:, 1:]."""
     x, t = wl.c4a(B=3, L=21, V=151936)
     xt, tt = upload(x), upload(t)
     zv, yv = xt[:, :-1], tt[:, 1:]
@@ -207,8 +213,11 @@ def test_long_rows_strided_3d_view(orc):
     check_oracle(orc, rf, dzf.reshape(-1, x.shape[-1]), z64, y, 0.5, 0.0, -100, "f32", "f32")
 
 
-def test_smem_rows_in_place_and_repeatable():
-    z, z32, y = wl.rows(300, 32000, "bf16", seed=9, std=2.0, ignore_frac=0.2)
+@pytest.mark.parametrize("V", [32000, 151936])
+def test_smem_rows_in_place_and_repeatable(V):
+    """Shared memory (32000) and L2 slices (151,936): two calls give the same
+    bits, and so does a call that writes dlogits over its own logits."""
+    z, z32, y = wl.rows(300, V, "bf16", seed=9, std=2.0, ignore_frac=0.2)
     zt, yt = upload(z, "bf16"), upload(y)
     g = torch.ones(1, device="cuda")
     r1, d1 = ce.ce_forward_backward(zt, yt, g, 0.1, return_argmax=True)
@@ -224,8 +233,11 @@ def test_smem_rows_in_place_and_repeatable():
     assert d3.data_ptr() == zc.data_ptr() and torch.equal(d1, zc)
 
 
-def test_smem_rows_bad_targets_and_nonfinite(orc):
-    N, V = 200, 40000
+@pytest.mark.parametrize("V", [20000, 40000])
+def test_smem_rows_bad_targets_and_nonfinite(orc, V):
+    """fp32 rows in shared memory (20000) and in L2 slices (40000, cluster of
+    2): bad and ignored targets, NaN, -inf and huge logits."""
+    N = 200
     rng = np.random.default_rng(7)
     z32 = rng.standard_normal((N, V)).astype(np.float32)
     y = rng.integers(0, V, size=N).astype(np.int32)
