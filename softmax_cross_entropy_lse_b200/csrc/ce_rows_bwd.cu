@@ -312,6 +312,40 @@ __global__ void __launch_bounds__(256, MINB) k_bwd_rows(BwdArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// dz of the vectors p * 32 + lane (p < P; all of them when FULL) of one
+// chunk staged in shared memory; TGT: the target column lies in the chunk,
+// dyc columns after its start.
+template <typename TI, typename TO, int P, bool FULL, bool TGT>
+__device__ __forceinline__ void ring_grad(const uint4* buf, int nvc, int lane, TO* dchunk, float2 nh,
+                                          float2 l2, float2 nl, float2 gg, float2 ne, float c_tgt,
+                                          int dyc) {
+    constexpr int VEC = ElemTraits<TI>::kVec;
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        const int vi = p * 32 + lane;
+        if (!FULL && vi >= nvc) continue;
+        float v[VEC], o[VEC];
+        unpack_words<TI>(buf[vi], v);
+#pragma unroll
+        for (int e = 0; e < VEC; e += 2) {
+            float2 d = __fadd2_rn(make_float2(v[e], v[e + 1]), nh);
+            d = __ffma2_rn(d, l2, nl);
+            const float2 pp = make_float2(ex2(d.x), ex2(d.y));
+            const float2 r2 = __ffma2_rn(gg, pp, ne);
+            o[e] = r2.x;
+            o[e + 1] = r2.y;
+        }
+        if constexpr (TGT) {
+            const int dy = dyc - vi * VEC;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e)
+                if (dy == e) o[e] -= c_tgt;
+        }
+        store_vec<TO, VEC>(dchunk, (int64_t)vi * VEC, 1, o);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Long rows through per-warp bulk-copy rings. A unit is (row, chunk of
 // vec_per_chunk vectors) and belongs to one warp; the warp's lane 0 keeps a
 // ring of kBRingStages 2 KB buffers filled with 1-D bulk copies issued ahead
@@ -445,35 +479,29 @@ __global__ void __launch_bounds__(kBRingWarps * 32, 2) k_bwd_ring(BwdArgs a) {
                 const int64_t left = nv - j * kBRingVecs;
                 const int nvc = (int)(left < kBRingVecs ? left : kBRingVecs);
                 const uint4* buf = reinterpret_cast<const uint4*>(ring + stage * kBRingVecs * 16);
-#pragma unroll
-                for (int p = 0; p < kPerLane; ++p) {
-                    const int vi = p * 32 + lane;
-                    if (vi >= nvc) continue;
-                    const int64_t col0 = (v0 + j * kBRingVecs + vi) * VEC;
+                const int64_t cc = (v0 + j * kBRingVecs) * VEC;  // first column of the chunk
+                TO* dchunk = drow + cc;
+                // the chunk that holds the target (one per row) takes its own
+                // warp-uniform branch; the others pay nothing for its term
+                const int64_t dyc = q.y - cc;
+                if (q.zero || q.bad) {
                     float o[VEC];
-                    if (q.zero || q.bad) {
 #pragma unroll
-                        for (int e = 0; e < VEC; ++e) o[e] = q.bad ? nan : 0.f;
-                    } else {
-                        float v[VEC];
-                        unpack_words<TI>(buf[vi], v);
+                    for (int e = 0; e < VEC; ++e) o[e] = q.bad ? nan : 0.f;
 #pragma unroll
-                        for (int e = 0; e < VEC; e += 2) {
-                            float2 d = __fadd2_rn(make_float2(v[e], v[e + 1]), nh);
-                            d = __ffma2_rn(d, l2, nl);
-                            const float2 pp = make_float2(ex2(d.x), ex2(d.y));
-                            const float2 r2 = __ffma2_rn(gg, pp, ne);
-                            o[e] = r2.x;
-                            o[e + 1] = r2.y;
-                        }
-                        const int64_t dy = q.y - col0;
-                        if (dy >= 0 && dy < VEC) {
-#pragma unroll
-                            for (int e = 0; e < VEC; ++e)
-                                if (e == dy) o[e] -= q.c_tgt;
-                        }
+                    for (int p = 0; p < kPerLane; ++p) {
+                        const int vi = p * 32 + lane;
+                        if (vi < nvc) store_vec<TO, VEC>(dchunk, (int64_t)vi * VEC, 1, o);
                     }
-                    store_vec<TO, VEC>(drow, col0, 1, o);
+                } else if (dyc >= 0 && dyc < (int64_t)nvc * VEC) {
+                    ring_grad<TI, TO, kPerLane, false, true>(buf, nvc, lane, dchunk, nh, l2, nl, gg, ne,
+                                                            q.c_tgt, (int)dyc);
+                } else if (nvc == kBRingVecs) {
+                    ring_grad<TI, TO, kPerLane, true, false>(buf, nvc, lane, dchunk, nh, l2, nl, gg, ne,
+                                                            q.c_tgt, 0);
+                } else {
+                    ring_grad<TI, TO, kPerLane, false, false>(buf, nvc, lane, dchunk, nh, l2, nl, gg, ne,
+                                                             q.c_tgt, 0);
                 }
             }
             fence_proxy_async_smem();
