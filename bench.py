@@ -732,7 +732,7 @@ def bench_linear(args, rk):
                    "parallelism": f"rows sharded over {world} rank(s), no data-path collective"},
         "e2e": {"value": round(world * step_flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": (N * D + V * D) * 2 + 4 * N, "d2h_bytes_per_step": 4 * N},
-        "gpu_launches": (2 + 1 + 4 * ((V + 8191) // 8192)) * args.steps,
+        "gpu_launches": (2 + 3 * ((V + 8191) // 8192)) * args.steps,
         "roofline": roofline("tensor", dom, achieved, peak_sust, src + " (sustained)",
                              recorded_traffic("c5", dom), dom_flop),
     }
