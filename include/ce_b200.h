@@ -148,12 +148,14 @@ ce_status ce_backward(const float* grad_out, int64_t grad_stride,
  * write, with the same definitions, readings and errors (argument meanings as
  * there). The logits cross HBM once instead of twice wherever a row fits on
  * chip: rows of up to 1024 elements stay in the registers of the lanes that
- * fold them; longer rows with 16-byte aligned, unit-stride rows (logits and
- * dlogits) and up to 4 x 112 KB per row are copied into shared memory, split
- * over a cluster of 1, 2 or 4 CTAs whose partial states meet once in
- * distributed shared memory, and differentiated from there. Those rows need
- * at least (number of SMs / cluster size) rows per call; otherwise, and for
- * longer or unaligned rows, the call runs the forward, then the backward.
+ * fold them. Longer rows need 16-byte aligned, unit-stride rows (logits and
+ * dlogits): rows of up to 112 KB are copied into one CTA's shared memory and
+ * differentiated from there; rows of up to 8 x 128 KB are split into slices
+ * over a cluster of 1 to 8 CTAs, whose partial states meet once in
+ * distributed shared memory, and each slice is read a second time from L1/L2
+ * for the gradient. Those rows need at least (number of SMs / cluster size)
+ * rows per call; otherwise, and for longer or unaligned rows, the call runs
+ * the forward, then the backward.
  * Sources: Ineshin, "A fused linear cross-entropy forward kernel for Apple
  * GPUs", section 1 (the backward needs only the row's log-sum-exp, which
  * the forward has just produced); MLX issue #4686 (the VJP).

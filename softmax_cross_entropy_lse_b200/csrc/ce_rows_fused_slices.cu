@@ -34,8 +34,8 @@
 // bits. The warp and CTA states of row i use exchange slots of parity i & 1,
 // so no slot is rewritten before every reader has passed the next barrier
 // (the race of Suryavanshi, "One barrier short", cannot occur). Every wait is
-// bounded; on expiry the kernel raises error bit 2, stops issuing copies,
-// drains those in flight and returns.
+// bounded; on expiry the kernel raises the timeout bit of the error word
+// (value 2), stops issuing copies, drains those in flight and returns.
 #include "ce_device.cuh"
 #include "ce_launch.h"
 #include "ce_sm100.cuh"
