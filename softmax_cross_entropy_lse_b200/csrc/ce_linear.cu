@@ -8,11 +8,18 @@
 // the logits tile by tile from the saved log-sum-exp.
 //
 // Design for B200 (not the page's Metal kernel):
-//  * one persistent GEMM engine, 128 x 256 output tiles, K in 64-element
-//    (128-byte) steps: a TMA producer warp fills a 4-stage shared-memory ring,
-//    one thread issues tcgen05.mma into a double-buffered f32 accumulator in
-//    tensor memory (2 x 256 columns), and four epilogue warps read the
-//    accumulator with tcgen05.ld, one TMEM lane (= one output row) per thread;
+//  * one persistent GEMM engine, K in 64-element (128-byte) steps: a TMA
+//    producer warp fills a shared-memory ring, one thread issues tcgen05.mma
+//    into a double-buffered f32 accumulator in tensor memory (2 x 256
+//    columns), and four epilogue warps read the accumulator with tcgen05.ld,
+//    one TMEM lane (= one output row) per thread. The forward runs one CTA
+//    per 128 x 256 tile (4 stages); the backward runs CTA pairs on 256 x 256
+//    tiles (6 stages, cta_group::2);
+//  * the CTAs in flight work on consecutive units. Row tiles run fastest when
+//    A is the operand that fits in L2 (H in the forward and in GEMM 1);
+//    column units run fastest in GEMMs 2 and 3, where B (H, or W_c) fits and
+//    A (G_c, 134 MB at N = 8192) does not, and B's lines then carry an
+//    evict_last L2 policy, so each B panel crosses DRAM once per launch;
 //  * forward epilogue: the online log-sum-exp of each row over a unit of
 //    consecutive vocabulary tiles, kept in registers, then a partial state
 //    per (unit, row) merged in unit order by a second launch;
@@ -38,6 +45,34 @@
 
 namespace ceb {
 using namespace sm100;
+
+// TMA loads with an L2 cache policy for the source lines (the engine marks the
+// operand that should stay in L2), and the policy itself.
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "l"(policy)
+        : "memory");
+}
+
+// An L2 policy under which the lines it marks are evicted after normal ones.
+__device__ __forceinline__ uint64_t l2_policy_keep() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void tma_load_2d_pair_hint(uint32_t dst, const CUtensorMap* map,
+                                                      uint32_t bar_cluster, int c0, int c1,
+                                                      uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "l"(policy)
+        : "memory");
+}
 
 constexpr int kBM = 128, kBN = 256, kBK = 64;
 constexpr uint32_t kABytes = kBM * kBK * 2;  // one CTA's A rows of a stage
@@ -78,6 +113,9 @@ struct GemmArgs {
     int tiles_per_unit;        // consecutive column tiles handled as one unit
     int n_units_n;             // ceil(n_nb / tiles_per_unit)
     int64_t units;             // n_mb * n_units_n
+    // unit order: row tiles fastest (0), or column units fastest (1), in which
+    // case B's lines are kept in L2 ahead of normal ones (see launch_gemm)
+    int n_fast;
     int kA0, kB0;              // K origin of A and B in their tensor maps
     unsigned int* err;
     unsigned long long wait_ns;  // limit of every pipeline wait
@@ -246,10 +284,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int s = 0;
             uint32_t ph = 0;
             uint32_t issued_mask = 0, last_ph = 0;  // per stage: has a load, its phase
+            const uint64_t pol_keep = l2_policy_keep();
             bool ok = true;
             for (int64_t u = u_first; u < a.units && ok; u += u_step) {
-                const int mb = (int)(u % a.n_mb);
-                const int un = (int)(u / a.n_mb);
+                const int mb = a.n_fast ? (int)(u / a.n_units_n) : (int)(u % a.n_mb);
+                const int un = a.n_fast ? (int)(u % a.n_units_n) : (int)(u / a.n_mb);
                 const int nb0 = un * a.tiles_per_unit;
                 const int nb1 = min(a.n_nb, nb0 + a.tiles_per_unit);
                 const int rowA = mb * Cfg::kTileM + (int)rank * kBM;
@@ -266,10 +305,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             if (lead) mbar_expect_tx(full_bar(s), CG * Cfg::kStageBytes);
                             const uint32_t fb = lead_full0 + 8u * s;
                             auto load = [&](uint32_t dst, const CUtensorMap* map, int c0, int c1) {
-                                if constexpr (CG == 1)
-                                    tma_load_2d(dst, map, fb, c0, c1);
-                                else
-                                    tma_load_2d_pair(dst, map, fb, c0, c1);
+                                if (a.n_fast && map == &tmB) {
+                                    if constexpr (CG == 1)
+                                        tma_load_2d_hint(dst, map, fb, c0, c1, pol_keep);
+                                    else
+                                        tma_load_2d_pair_hint(dst, map, fb, c0, c1, pol_keep);
+                                } else {
+                                    if constexpr (CG == 1)
+                                        tma_load_2d(dst, map, fb, c0, c1);
+                                    else
+                                        tma_load_2d_pair(dst, map, fb, c0, c1);
+                                }
                             };
                             const int k0a = a.kA0 + kb * kBK, k0b = a.kB0 + kb * kBK;
                             if constexpr (AMN) {
@@ -322,7 +368,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             uint32_t ph = 0, it = 0;
             bool ok = true;
             for (int64_t u = u_first; u < a.units && ok; u += u_step) {
-                const int un = (int)(u / a.n_mb);
+                const int un = a.n_fast ? (int)(u % a.n_units_n) : (int)(u / a.n_mb);
                 const int nb0 = un * a.tiles_per_unit;
                 const int nb1 = min(a.n_nb, nb0 + a.tiles_per_unit);
                 for (int nb = nb0; nb < nb1 && ok; ++nb, ++it) {
@@ -388,8 +434,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t it = 0;
         bool ok = true;
         for (int64_t u = u_first; u < a.units && ok; u += u_step) {
-            const int mb = (int)(u % a.n_mb);
-            const int un = (int)(u / a.n_mb);
+            const int mb = a.n_fast ? (int)(u / a.n_units_n) : (int)(u % a.n_mb);
+            const int un = a.n_fast ? (int)(u % a.n_units_n) : (int)(u / a.n_mb);
             const int nb0 = un * a.tiles_per_unit;
             const int nb1 = min(a.n_nb, nb0 + a.tiles_per_unit);
             const int64_t m = (int64_t)mb * Cfg::kTileM + (int64_t)rank * kBM + r_in_tile;
@@ -818,6 +864,7 @@ ce_status linear_ce_backward(const float* grad_out, int64_t grad_stride, const v
             a.C = static_cast<uint8_t*>(dW) + (size_t)v0 * D * esz;
             a.ldc = D;
             a.c_f32 = dW_dt == CE_F32;
+            a.n_fast = 1;  // H (B) stays in L2 while the G_c panels stream
             if (launch_gemm<kEpiStore, kCgBwd, true, true>(mGmn, mHmn, a, sms, s) != cudaSuccess)
                 return CE_ECUDA;
         }
@@ -842,6 +889,7 @@ ce_status linear_ce_backward(const float* grad_out, int64_t grad_stride, const v
             a.C = dH;
             a.ldc = D;
             a.c_f32 = dH_dt == CE_F32;
+            a.n_fast = 1;  // W_c (B) stays in L2 while the G_c panels stream
             if (launch_gemm<kEpiAccum, kCgBwd, false, true>(mG, mWmn, a, sms, s) != cudaSuccess)
                 return CE_ECUDA;
         }
