@@ -40,7 +40,10 @@
 #include "ce_launch.h"
 #include "ce_sm100.cuh"
 
-#include <atomic>
+#include <mutex>
+#include <utility>
+#include <vector>
+
 
 namespace ceb {
 
@@ -441,26 +444,30 @@ static cudaError_t launch_slices_k(const SliceRowPlan& sp, const FusedArgs& a, c
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = CL > 1 ? 1 : 0;
-    // co-resident clusters (CTAs when CL = 1) for this shared-memory size,
-    // cached per size
-    static std::atomic<long long> cached{0};  // (smem << 20) | clusters
-    const long long c = cached.load(std::memory_order_relaxed);
+    // co-resident clusters (CTAs when CL = 1), cached per (device, shared memory)
     int clusters = 0;
-    if (c != 0 && (size_t)(c >> 20) == smem) {
-        clusters = (int)(c & 0xfffff);
-    } else {
-        cudaError_t e;
-        if constexpr (CL > 1) {
-            cfg.gridDim = dim3(CL * sp.sms);
-            e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
-        } else {
-            int per_sm = 0;
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSmWarps * 32, smem);
-            clusters = per_sm * sp.sms;
-        }
+    if constexpr (CL > 1) {
+        // smem is 0 here: the cache keyed by (kernel, device) fits
+        const cudaError_t e = max_active_clusters((const void*)kern, cfg, &clusters);
         if (e != cudaSuccess) return e;
-        if (clusters < 1) return cudaErrorInvalidConfiguration;
-        cached.store(((long long)smem << 20) | clusters, std::memory_order_relaxed);
+    } else {
+        static std::mutex mu;
+        static std::vector<std::pair<long long, int>> cache;  // ((device << 32) | smem, CTAs)
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+        const long long key = ((long long)dev << 32) | (long long)smem;
+        std::lock_guard<std::mutex> lock(mu);
+        for (const auto& c : cache)
+            if (c.first == key) clusters = c.second;
+        if (clusters == 0) {
+            int per_sm = 0;
+            const cudaError_t e =
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSmWarps * 32, smem);
+            if (e != cudaSuccess) return e;
+            clusters = per_sm * sp.sms;
+            if (clusters < 1) return cudaErrorInvalidConfiguration;
+            cache.emplace_back(key, clusters);
+        }
     }
     const int64_t want = a.f.N < clusters ? a.f.N : clusters;
     cfg.gridDim = dim3((unsigned)(want * CL));
