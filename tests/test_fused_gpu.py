@@ -156,6 +156,8 @@ def _padded(N, V, pad, dtype, seed, std=2.0, ignore_frac=0.1):
     (100000, 80, "f32"),       # L2 slices, cluster of 4, fp32
     (151936, 40, "f32"),       # L2 slices, cluster of 8 (608 KB rows)
     (151936, 30, "bf16"),      # too few rows for every SM: the forward, then the VJP
+    (524288, 24, "bf16"),      # the largest L2-slice row: 8 slices of exactly 128 KB
+    (524296, 24, "bf16"),      # one vector more: the forward, then the VJP
     (600000, 12, "bf16"),      # beyond 8 slices of 128 KB: the forward, then the VJP
 ])
 def test_smem_rows_vs_oracle(orc, V, N, dt):
