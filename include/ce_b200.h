@@ -68,7 +68,7 @@ typedef enum {
     CE_EWORKSPACE = 3, /* workspace missing or smaller than the *_workspace_size query */
     CE_ECUDA = 4,      /* a CUDA runtime call failed (launch, attribute query) */
     CE_ETARGET = 5,    /* device flag: a target outside [0, V) that is not ignore_index */
-    CE_ENOTSUP = 6,    /* a configuration this build does not implement */
+    CE_ENOTSUP = 6,    /* a configuration the library does not implement */
     CE_ETIMEOUT = 7    /* device flag: a kernel gave up a bounded wait (outputs invalid) */
 } ce_status;
 
