@@ -622,8 +622,9 @@ __device__ __forceinline__ OnlineState shfl_xor_state(const OnlineState& st, int
 // group takes its max first, every lane rescales its own (s, t) to it once,
 // and the rescaled terms are summed along the butterfly: the same merge
 // operator, with one exponential per lane instead of two per round. WITH_T =
-// false reduces (m, s) only (t and k are left as they are).
-template <int G, bool ARGMAX, bool WITH_T = true>
+// false reduces (m, s) only (t and k are left as they are); WITH_K = false
+// leaves the count k unreduced, for a last merge whose caller reads only t.
+template <int G, bool ARGMAX, bool WITH_T = true, bool WITH_K = true>
 __device__ __forceinline__ void group_reduce(OnlineState& st) {
     if constexpr (ARGMAX) {
 #pragma unroll
@@ -648,7 +649,7 @@ __device__ __forceinline__ void group_reduce(OnlineState& st) {
             s += __shfl_xor_sync(0xffffffffu, s, off);
             if constexpr (WITH_T) {
                 t += __shfl_xor_sync(0xffffffffu, t, off);
-                k += __shfl_xor_sync(0xffffffffu, k, off);
+                if constexpr (WITH_K) k += __shfl_xor_sync(0xffffffffu, k, off);
             }
         }
         st.m = M;
@@ -711,7 +712,8 @@ __device__ __forceinline__ void finalize_row(const OnlineState& st, float zy, in
         atomicOr(o.err, 1u);
     } else {
         loss = L - (1.f - eps) * (zy - st.m);
-        if (eps != 0.f) loss -= eps * (st.t / (float)V);
+        // t / V as t times 1/V: a kernel's rows share the reciprocal
+        if (eps != 0.f) loss -= eps * (st.t * (1.0f / (float)V));
     }
     o.loss[r] = loss;
     if (write_argmax) o.argmax[r] = st.ai < 0 ? 0 : st.ai;

@@ -176,7 +176,8 @@ __global__ void __launch_bounds__(kPipeWarps * 32, MINB) k_fwd_packed_pipe(FwdAr
                 if constexpr (ARGMAX) argmax_vecs<U, VEC, true>(st, v, ok, c0);
             }
         }
-        group_reduce<G, ARGMAX>(st);
+        // the last merge of the row: finalize_row reads t, not the count
+        group_reduce<G, ARGMAX, true, false>(st);
         if (active && gl == 0) finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);
     }
     cp_async_wait<0>();
