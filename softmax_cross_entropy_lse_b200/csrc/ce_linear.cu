@@ -15,11 +15,11 @@
 //    one TMEM lane (= one output row) per thread. The forward runs one CTA
 //    per 128 x 256 tile (4 stages); the backward runs CTA pairs on 256 x 256
 //    tiles (6 stages, cta_group::2);
-//  * the CTAs in flight work on consecutive units. Row tiles run fastest when
-//    A is the operand that fits in L2 (H in the forward and in GEMM 1);
-//    column units run fastest in GEMMs 2 and 3, where B (H, or W_c) fits and
-//    A (G_c, 134 MB at N = 8192) does not, and B's lines then carry an
-//    evict_last L2 policy, so each B panel crosses DRAM once per launch;
+//  * the CTAs in flight work on consecutive units. Row tiles run fastest, so
+//    the row operand A stays in L2 (H in the forward and in GEMM 1); in GEMMs
+//    2 and 3, when A (G_c, 134 MB at N = 8192) is the larger operand, column
+//    units run fastest instead and B's lines (H, or W_c) carry an evict_last
+//    L2 policy, so each B panel crosses DRAM once per launch;
 //  * forward epilogue: the online log-sum-exp of each row over a unit of
 //    consecutive vocabulary tiles, kept in registers, then a partial state
 //    per (unit, row) merged in unit order by a second launch;
@@ -864,7 +864,9 @@ ce_status linear_ce_backward(const float* grad_out, int64_t grad_stride, const v
             a.C = static_cast<uint8_t*>(dW) + (size_t)v0 * D * esz;
             a.ldc = D;
             a.c_f32 = dW_dt == CE_F32;
-            a.n_fast = 1;  // H (B) stays in L2 while the G_c panels stream
+            // the smaller operand stays in L2 while the other streams: H (B)
+            // when G_c (A, vcv x N) is the larger
+            a.n_fast = vcv > D ? 1 : 0;
             if (launch_gemm<kEpiStore, kCgBwd, true, true>(mGmn, mHmn, a, sms, s) != cudaSuccess)
                 return CE_ECUDA;
         }
@@ -889,7 +891,8 @@ ce_status linear_ce_backward(const float* grad_out, int64_t grad_stride, const v
             a.C = dH;
             a.ldc = D;
             a.c_f32 = dH_dt == CE_F32;
-            a.n_fast = 1;  // W_c (B) stays in L2 while the G_c panels stream
+            // W_c (B, vcv x D) stays in L2 when G_c (A, N x vcv) is the larger
+            a.n_fast = N > D ? 1 : 0;
             if (launch_gemm<kEpiAccum, kCgBwd, false, true>(mG, mWmn, a, sms, s) != cudaSuccess)
                 return CE_ECUDA;
         }
