@@ -222,7 +222,8 @@ __global__ void __launch_bounds__(kSmWarps * 32, (SliceShape<ARGMAX, GL>::kMinBl
     __shared__ __align__(8) uint64_t full_bar[kSmMaxChunks];
     __shared__ OnlineState wslot[2][kSmWarps];
     // CTA states of the cluster, pushed by their owners: [row parity][source
-    // rank][two 16-byte words], completed on xbar[row parity]
+    // rank][two 16-byte words: (m, s, t, k), (argmax value, argmax index, z_y
+    // if the target lies in the source's slice, 0)], completed on xbar[row parity]
     __shared__ __align__(16) uint4 xslot[2][CL][2];
     __shared__ __align__(8) uint64_t xbar[2];
     __shared__ int abort_flag;
@@ -286,8 +287,16 @@ __global__ void __launch_bounds__(kSmWarps * 32, (SliceShape<ARGMAX, GL>::kMinBl
         const bool ign = y == a.ignore;
         const bool bad = !ign && (y < 0 || y >= a.V);
         const int64_t yc = (ign || bad) ? -1 : y;
+        // z_y is read by the CTA whose slice holds it, before that CTA's own
+        // gradient pass can overwrite it (dlogits may be the logits), and
+        // travels to the first CTA with that CTA's state
+        int owner = 0;
+        if (CL > 1 && yc >= 0) {
+            const int64_t yv = yc / VEC;
+            owner = yv >= nvec ? CL - 1 : (int)min((int64_t)(CL - 1), yv / sp.vec_per_cta);
+        }
         float zy = 0.f;
-        if (rank == 0 && tid == 0 && yc >= 0) zy = to_f32(row[yc]);
+        if (rank == (uint32_t)owner && tid == 0 && yc >= 0) zy = to_f32(row[yc]);
 
         // ---- forward: fold the slice (from global memory, or from shared
         // memory as its chunks land)
@@ -340,7 +349,7 @@ __global__ void __launch_bounds__(kSmWarps * 32, (SliceShape<ARGMAX, GL>::kMinBl
                 mbar_expect_tx(bar, (uint32_t)(CL - 1) * 32u);
                 const uint4 w0 = make_uint4(__float_as_uint(st.m), __float_as_uint(st.s),
                                             __float_as_uint(st.t), (uint32_t)st.k);
-                const uint4 w1 = make_uint4(__float_as_uint(st.av), (uint32_t)st.ai, 0u, 0u);
+                const uint4 w1 = make_uint4(__float_as_uint(st.av), (uint32_t)st.ai, __float_as_uint(zy), 0u);
                 const uint32_t src = smem_u32(&xslot[par][rank][0]);
 #pragma unroll
                 for (uint32_t k = 0; k < (uint32_t)CL; ++k) {
@@ -362,6 +371,7 @@ __global__ void __launch_bounds__(kSmWarps * 32, (SliceShape<ARGMAX, GL>::kMinBl
                 st.ai = (int)w1.y;
             }
             group_reduce<CL, ARGMAX, WITH_T>(st);
+            if (rank == 0 && tid == 0 && owner != 0) zy = __uint_as_float(xslot[par][owner][1].z);
         }
         if (rank == 0 && tid == 0) finalize_row(st, zy, y, a.ignore, a.V, a.eps, out, r, ARGMAX);
 
