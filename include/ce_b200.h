@@ -337,10 +337,11 @@ ce_status ce_forward_noalloc(const void* logits, ce_dtype dt, ce_layout lg,
 ce_status ce_get_error(void* cuda_stream);
 
 /* Testing hook for the bounded waits; the pages have no counterpart. Sets the
- * wait limit of the GEMM engine and of the long-row forward's bulk-copy ring
- * for the launches this process makes afterwards (limit_ns = 0 restores the
- * default of 2 s). With starve = 1 those launches issue none of their copies,
- * so every wait for data runs out after the limit: tests use it to check that
+ * wait limit of the GEMM engine, of the long-row forward's bulk-copy ring and
+ * of ce_forward_backward's long-row slices for the launches this process makes
+ * afterwards (limit_ns = 0 restores the default of 2 s). With starve = 1 those
+ * launches issue none of their copies (and the slices push no state to their
+ * cluster peers), so every wait for data runs out after the limit: tests use it to check that
  * a wait that runs out ends the kernel with CE_ETIMEOUT and leaves the
  * context and the next call correct. starve = 0 is normal operation; any
  * other value is CE_EINVAL. Not for production use: a starved launch writes

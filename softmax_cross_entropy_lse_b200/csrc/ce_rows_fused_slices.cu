@@ -268,8 +268,10 @@ __global__ void __launch_bounds__(kSmWarps * 32, (SliceShape<ARGMAX, GL>::kMinBl
     };
 
     // bit i of the masks: this warp's i-th chunk (c = wid + 8 i)
+    // (a starved launch, a testing mode, copies nothing and pushes no state:
+    // its waits run out)
     uint32_t pend = 0, phase = 0;
-    if (!GL && cid < a.N) {
+    if (!GL && cid < a.N && !a.starve) {
         for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps) {
             if (lane == 0) issue(cid, c);
             pend |= 1u << i;
@@ -314,7 +316,7 @@ __global__ void __launch_bounds__(kSmWarps * 32, (SliceShape<ARGMAX, GL>::kMinBl
         }
         for (int i = 0, c = wid; !GL && c < nch; ++i, c += kSmWarps) {
             if (!dead) {
-                if (mbar_wait(smem_u32(&full_bar[c]), (phase >> i) & 1u, &abort_flag)) {
+                if (mbar_wait(smem_u32(&full_bar[c]), (phase >> i) & 1u, &abort_flag, a.wait_ns)) {
                     phase ^= 1u << i;
                     pend &= ~(1u << i);
                 } else {
@@ -353,13 +355,13 @@ __global__ void __launch_bounds__(kSmWarps * 32, (SliceShape<ARGMAX, GL>::kMinBl
                 const uint32_t src = smem_u32(&xslot[par][rank][0]);
 #pragma unroll
                 for (uint32_t k = 0; k < (uint32_t)CL; ++k) {
-                    if (k == rank) continue;
+                    if (k == rank || a.starve) continue;
                     const uint32_t ra = mapa_shared(src, k), rb = mapa_shared(bar, k);
                     st_async_v4(ra, w0, rb);
                     st_async_v4(ra + 16, w1, rb);
                 }
             }
-            if (!dead && !mbar_wait(bar, (uint32_t)(it >> 1) & 1u, &abort_flag)) dead = true;
+            if (!dead && !mbar_wait(bar, (uint32_t)(it >> 1) & 1u, &abort_flag, a.wait_ns)) dead = true;
             const uint32_t from = (uint32_t)(lane & (CL - 1));
             if (from != rank) {
                 const uint4 w0 = xslot[par][from][0], w1 = xslot[par][from][1];
@@ -400,7 +402,7 @@ __global__ void __launch_bounds__(kSmWarps * 32, (SliceShape<ARGMAX, GL>::kMinBl
         // (one proxy fence for all of them)
         if constexpr (!GL) fence_proxy_async_smem();
         __syncwarp();
-        if (!GL && rn < a.N && !dead) {
+        if (!GL && rn < a.N && !dead && !a.starve) {
             for (int i = 0, c = wid; c < nch; ++i, c += kSmWarps) {
                 if (lane == 0) issue(rn, c);
                 pend |= 1u << i;
@@ -481,7 +483,11 @@ static cudaError_t launch_slices_k(const SliceRowPlan& sp, const FusedArgs& a, c
     }
     const int64_t want = a.f.N < clusters ? a.f.N : clusters;
     cfg.gridDim = dim3((unsigned)(want * CL));
-    return cudaLaunchKernelEx(&cfg, kern, a, sp);
+    FusedArgs b = a;  // the wait limit and the testing hook's starve flag
+    const WaitPolicy wp = wait_policy();
+    b.f.wait_ns = wp.limit_ns;
+    b.f.starve = wp.starve;
+    return cudaLaunchKernelEx(&cfg, kern, b, sp);
 }
 
 // Shared-memory slices run one CTA per row; L2 slices take clusters of 1 to 8.

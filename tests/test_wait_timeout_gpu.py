@@ -2,8 +2,9 @@
 with an error status, and the context stays usable.
 
 The kernels that stream their operands through mbarrier pipelines (the
-tensor-core GEMM engine of the fused-linear calls and the bulk-copy ring of
-the long-row forward) give up a wait after a time limit, raise the timeout
+tensor-core GEMM engine of the fused-linear calls, the bulk-copy ring of the
+long-row forward, and the slices of the one-call forward + VJP, which also
+wait on their cluster peers' states) give up a wait after a time limit, raise the timeout
 bit of the device error word, let the copies and MMAs they started complete,
 free their tensor memory and return. These tests make such a wait run out
 without any fault: the testing hook sets a short limit and starves the
@@ -94,6 +95,26 @@ def test_bulk_copy_ring_wait_runs_out(orc):
     rt, at = loss_tol("bf16")
     assert_close(f32(r.loss), loss, rt, at, "loss after a timeout")
     assert_close(f32(r.lse), lse, rt, at, "lse after a timeout")
+
+
+@pytest.mark.parametrize("N,V", [(600, 32000), (160, 151936)])
+def test_fused_slices_wait_runs_out(orc, N, V):
+    """The one-call forward + VJP of long rows: 32000-wide rows wait for their
+    bulk copies into shared memory, 151,936-wide rows (L2 slices over a 4-CTA
+    cluster) for the states their peers push; starved, both waits run out."""
+    z, z32, y = wl.rows(N, V, "bf16", seed=14, std=2.0)
+    zt, yt = upload(z, "bf16"), upload(y)
+    g = torch.ones(1, device="cuda")
+    good_r, good_dz = ce.ce_forward_backward(zt, yt, g)
+    assert ce.get_error() == 0
+    assert starved(lambda: ce.ce_forward_backward(zt, yt, g)) == CE_ETIMEOUT
+    r, dz = ce.ce_forward_backward(zt, yt, g)
+    assert ce.get_error() == 0
+    assert torch.equal(r.loss, good_r.loss) and torch.equal(r.lse, good_r.lse)
+    assert torch.equal(dz, good_dz)
+    loss, lse, _ = orc.ce_forward(z32.astype(np.float64), y)
+    rt, at = loss_tol("bf16")
+    assert_close(f32(r.loss), loss, rt, at, "loss after a timeout")
 
 
 def test_timeout_outranks_bad_target():
